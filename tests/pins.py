@@ -1,0 +1,237 @@
+"""Pins for the oracle: checks against what the pages and the mathematics fix.
+
+Every check takes the implementation under test as arguments, so that
+test_oracle_mutations.py can run the same checks on deliberately broken copies of
+the oracle and show that each planted mistake is caught.  A check returns None
+when it passes and raises AssertionError otherwise.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from golden_loader import load
+from oracle import brute
+
+TOL = 1e-12
+
+
+def _close(a, b, tol=TOL, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, (what, a.shape, b.shape)
+    same_inf = (np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b)))
+    diff = np.where(same_inf, 0.0, np.abs(a - b))
+    assert np.all(np.isfinite(diff)), (what, a, b)
+    m = float(diff.max(initial=0.0))
+    scale = max(1.0, float(np.abs(np.where(np.isinf(b), 0, b)).max(initial=0.0)))
+    assert m <= tol * scale, f"{what}: max diff {m}"
+
+
+# ---------------------------------------------------------------- definition
+
+def check_golden_attend(attend):
+    for name in ("attend_two_keys.txt", "attend_three_keys_scaled.txt"):
+        g = load(name)
+        d = len(g["q"])
+        dv = len(g["A"])
+        q = g["q"].reshape(1, d)
+        k = g["k"].reshape(-1, d)
+        v = g["v"].reshape(-1, dv)
+        a, l = attend(q, k, v, float(g["scale"][0]))
+        _close(a[0], g["A"], what=name + " A")
+        _close(l[0], g["L"][0], what=name + " L")
+
+
+def check_brute_force(attend, seed=0):
+    """Random tiny inputs with n != m != d != dv, mild and sharp scores."""
+    rng = np.random.default_rng(seed)
+    for (n, m, d, dv, sharp) in [(3, 5, 4, 6, 1.0), (1, 1, 3, 2, 1.0), (4, 7, 2, 3, 6.0), (2, 9, 5, 5, 0.05)]:
+        q = rng.standard_normal((n, d)) * sharp
+        k = rng.standard_normal((m, d)) * sharp
+        v = rng.standard_normal((m, dv))
+        scale = 1.0 / math.sqrt(d)
+        a, l = attend(q, k, v, scale)
+        for i in range(n):
+            ab, lb = brute.attend_one(list(q[i]), [list(x) for x in k], [list(x) for x in v], scale)
+            _close(a[i], ab, tol=1e-12, what="brute A")
+            _close(l[i], lb, tol=1e-12, what="brute L")
+
+
+def check_closed_forms(attend, seed=1):
+    rng = np.random.default_rng(seed)
+    d, dv = 6, 4
+    # one key: A = v, L = s
+    q = rng.standard_normal((3, d)); k = rng.standard_normal((1, d)); v = rng.standard_normal((1, dv))
+    a, l = attend(q, k, v, 0.7)
+    _close(a, np.repeat(v, 3, axis=0), what="one key A")
+    _close(l, 0.7 * (q @ k[0]), what="one key L")
+    # all scores equal (q = 0): A = mean(V), L = ln m
+    m = 11
+    k = rng.standard_normal((m, d)); v = rng.standard_normal((m, dv))
+    a, l = attend(np.zeros((2, d)), k, v, 0.3)
+    _close(a, np.repeat(v.mean(axis=0, keepdims=True), 2, axis=0), what="uniform A")
+    _close(l, np.full(2, math.log(m)), what="uniform L")
+    # constant values: A = c
+    q = rng.standard_normal((4, d)) * 3
+    vc = np.tile(np.array([[1.5, -2.0, 0.25, 7.0]]), (m, 1))
+    a, _ = attend(q, k, vc, 0.5)
+    _close(a, np.tile(vc[:1], (4, 1)), what="constant V")
+    # adding c to every score: A unchanged, L shifted by c
+    c = 2.75
+    q1 = np.concatenate([q, np.ones((4, 1))], axis=1)
+    k1 = np.concatenate([k, np.full((m, 1), c / 0.5)], axis=1)
+    a0, l0 = attend(q, k, v, 0.5)
+    a1, l1 = attend(q1, k1, v, 0.5)
+    _close(a1, a0, what="shift A")
+    _close(l1, l0 + c, what="shift L")
+    # empty key set: A = 0, L = -inf
+    a, l = attend(q, np.zeros((0, d)), np.zeros((0, dv)), 0.5)
+    _close(a, np.zeros((4, dv)), what="empty A")
+    assert np.all(np.isneginf(l)), "empty L"
+
+
+# ---------------------------------------------------------------- merge
+
+def check_golden_merge(merge):
+    g = load("merge_two_partials.txt")
+    a, l = merge(g["a_out"][None], g["l_out"], g["a_in"][None], g["l_in"])
+    _close(a[0], g["A"], what="golden merge A")
+    _close(l[0], g["L"][0], what="golden merge L")
+    g = load("merge_empty_side.txt")
+    a, l = merge(g["a_out"][None], g["l_out"], g["a_in"][None], g["l_in"])
+    _close(a[0], g["A"], what="empty side A")
+    _close(l[0], g["L"][0], what="empty side L")
+    a, l = merge(g["a_out"][None], np.array([-np.inf]), g["a_in"][None], np.array([-np.inf]))
+    _close(a[0], g["both_A"], what="both empty A")
+    assert np.isneginf(l[0]), "both empty L"
+    # and symmetrically with the empty side second
+    a, l = merge(g["a_in"][None], g["l_in"], g["a_out"][None], g["l_out"])
+    _close(a[0], g["A"], what="empty side (swapped) A")
+
+
+def check_fresh_cache_identity(attend, merge, seed=2):
+    """merge(attend(Q, J_out), attend(Q, J_in)) == attend(Q, J_out U J_in)."""
+    rng = np.random.default_rng(seed)
+    for (n, m1, m2, d, sharp) in [(5, 13, 4, 8, 1.0), (3, 1, 9, 4, 5.0), (2, 30, 30, 16, 0.2)]:
+        q = rng.standard_normal((n, d)) * sharp
+        k1 = rng.standard_normal((m1, d)); v1 = rng.standard_normal((m1, 3))
+        k2 = rng.standard_normal((m2, d)) * sharp; v2 = rng.standard_normal((m2, 3))
+        s = 1 / math.sqrt(d)
+        ao, lo = attend(q, k1, v1, s)
+        ai, li = attend(q, k2, v2, s)
+        a, l = merge(ao, lo, ai, li)
+        af, lf = attend(q, np.concatenate([k1, k2]), np.concatenate([v1, v2]), s)
+        _close(a, af, what="fresh identity A")
+        _close(l, lf, what="fresh identity L")
+
+
+def check_merge_order_independent(attend, merge, seed=3):
+    """Any partition of the keys into 2..16 chunks, merged in any order and tree
+    shape, gives the same (A, L) as one attention over all keys."""
+    rng = np.random.default_rng(seed)
+    n, m, d = 4, 64, 8
+    q = rng.standard_normal((n, d)) * 2
+    k = rng.standard_normal((m, d)); v = rng.standard_normal((m, 5))
+    s = 1 / math.sqrt(d)
+    af, lf = attend(q, k, v, s)
+    for trial in range(12):
+        nchunks = int(rng.integers(2, 17))
+        cuts = np.sort(rng.choice(np.arange(1, m), size=nchunks - 1, replace=False))
+        bounds = np.concatenate([[0], cuts, [m]])
+        parts = [attend(q, k[a:b], v[a:b], s) for a, b in zip(bounds[:-1], bounds[1:])]
+        # include an empty chunk now and then
+        if trial % 3 == 0:
+            parts.append(attend(q, k[:0], v[:0], s))
+        order = rng.permutation(len(parts))
+        parts = [parts[i] for i in order]
+        while len(parts) > 1:                     # random tree shape
+            i = int(rng.integers(0, len(parts) - 1))
+            (a1, l1), (a2, l2) = parts[i], parts[i + 1]
+            parts[i:i + 2] = [merge(a1, l1, a2, l2)]
+        a, l = parts[0]
+        _close(a, af, tol=1e-11, what="tree merge A")
+        _close(l, lf, tol=1e-11, what="tree merge L")
+    # commutativity, exactly
+    a1, l1 = attend(q, k[:20], v[:20], s)
+    a2, l2 = attend(q, k[20:], v[20:], s)
+    x = merge(a1, l1, a2, l2)
+    y = merge(a2, l2, a1, l1)
+    _close(x[0], y[0], tol=1e-15, what="commutative A")
+    _close(x[1], y[1], tol=1e-15, what="commutative L")
+
+
+# ---------------------------------------------------------------- gates
+
+def check_golden_gates(decide):
+    g = load("gates.txt")
+    tc = g["tau_cases"].reshape(-1, 3)
+    for tau, m, exp in tc:
+        rec = decide(1, int(tau), 0.0, np.ones((1, 1), bool), np.array([int(m)]), None, None)
+        assert bool(rec[0, 0]) == bool(exp), ("tau", tau, m, exp)
+    gc = g["gamma_cases"].reshape(-1, 3)
+    for gamma, cos, exp in gc:
+        rec = decide(2, 0, float(gamma), np.ones((1, 1), bool), np.array([0]), np.array([[cos]]), None)
+        assert bool(rec[0, 0]) == bool(exp), ("gamma", gamma, cos, exp)
+    # an invalid cache always recomputes, even under forced reuse
+    rec = decide(8, 0, 0.0, np.zeros((1, 2), bool), np.array([0]), None, None)
+    assert rec.all(), "invalid cache must recompute"
+    rec = decide(4, 100, 0.0, np.ones((1, 2), bool), np.array([0]), None, None)
+    assert rec.all(), "force recompute"
+    rec = decide(8 | 1, 4, 0.0, np.ones((1, 2), bool), np.array([99]), None, None)
+    assert not rec.any(), "force reuse overrides a failing tau gate"
+    # both gates: AND on reuse
+    rec = decide(3, 4, 0.5, np.ones((2, 2), bool), np.array([3, 3]), np.array([[0.9, 0.1], [0.6, 0.7]]), None)
+    assert rec.tolist() == [[False, True], [False, False]], rec
+    rec = decide(3, 4, 0.5, np.ones((1, 2), bool), np.array([4]), np.array([[0.9, 0.9]]), None)
+    assert rec.all(), "tau failure must recompute regardless of cos"
+
+
+def check_cosine(head_cosine):
+    """cos(x, x) = 1, cos(x, -x) = -1, cos(x, 2x) = 1, orthogonal rows = 0, over the
+    active rows of each sequence only (cache rows addressed by block position)."""
+    from cached_split_attention_b200.workloads import make_problem
+    p = make_problem([[0, 2], [1]], [3, 3], [3, 2], 2, 1, 4)
+    q = np.zeros((3, 2, 4))
+    q_ref = np.zeros((5, 2, 4))
+    # seq 0 rows at block positions 0 and 2 -> cache rows 0 and 2
+    x = np.array([[1.0, 2.0, 0.0, -1.0], [0.5, 0.0, 3.0, 1.0]])
+    q[0:2, 0] = x
+    q_ref[[0, 2], 0] = x
+    q[0:2, 1] = x
+    q_ref[[0, 2], 1] = -2.0 * x
+    q_ref[1, 0] = 100.0            # an inactive position: must be ignored
+    # seq 1: row at block position 1 -> cache row 3 + 1 = 4
+    q[2, 0] = [1, 0, 0, 0]
+    q_ref[4, 0] = [0, 1, 0, 0]
+    q[2, 1] = [1, 1, 0, 0]
+    q_ref[4, 1] = [3, 3, 0, 0]
+    cos = head_cosine(p, q, q_ref)
+    _close(cos, np.array([[1.0, -1.0], [0.0, 1.0]]), tol=1e-15, what="cosine")
+
+
+# ---------------------------------------------------------------- problem-level
+
+def check_problem_vs_brute(attend_problem, merge, attend_full_fn=None, seed=4):
+    """A GQA varlen problem (3 sequences, ragged, one with an empty prefix): the
+    split partials merged must equal brute-force full attention over J_out U J_in."""
+    from cached_split_attention_b200.workloads import make_problem, normal_bf16
+    from oracle.attention import bf16_to_f64
+    rng = np.random.default_rng(seed)
+    Hq, Hk, d = 4, 2, 8
+    p = make_problem([[0, 1, 2], [1, 3], [0]], [5, 0, 3], [3, 4, 2], Hq, Hk, d)
+    q = normal_bf16(rng, (p.total_q, Hq, d), 1.5)
+    ko = normal_bf16(rng, (p.total_kv_out, Hk, d)); vo = normal_bf16(rng, (p.total_kv_out, Hk, d))
+    ki = normal_bf16(rng, (p.total_kv_in, Hk, d)); vi = normal_bf16(rng, (p.total_kv_in, Hk, d))
+    ao, lo = attend_problem(p, q, ko, vo, "out")
+    ai, li = attend_problem(p, q, ki, vi, "in")
+    a, l = merge(ao, lo, ai, li)
+    tolist = lambda x: bf16_to_f64(x).tolist()
+    ab, lb = brute.attend_full_problem(p, tolist(q), tolist(ko), tolist(vo), tolist(ki), tolist(vi))
+    _close(a, np.array(ab), what="problem A")
+    _close(l, np.array(lb), what="problem L")
+    if attend_full_fn is not None:
+        af, lf = attend_full_fn(p, q, ko, vo, ki, vi)
+        _close(af, np.array(ab), what="attend_full A")
+        _close(lf, np.array(lb), what="attend_full L")

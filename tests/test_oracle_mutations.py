@@ -1,0 +1,122 @@
+"""Plant plausible mistakes in copies of the oracle and show that a pin fails.
+
+Each mutant is the oracle function's own source with one edit (a dropped term, a
+wrong sign, a wrong axis or index, a relaxed comparison), compiled into a private
+namespace; the real oracle is never modified.  Every mutant must make at least one
+of the pin checks in pins.py fail, otherwise the pins would not be able to tell the
+oracle from a broken one.
+"""
+import inspect
+import textwrap
+
+import pytest
+
+import pins
+from oracle import attention, policy
+
+
+def mutate(module, name, old, new, extra=None):
+    src = textwrap.dedent(inspect.getsource(getattr(module, name)))
+    assert src.count(old) >= 1, (name, old)
+    src = src.replace(old, new, 1)
+    ns = dict(vars(module))
+    if extra:
+        ns.update(extra)
+    exec(compile(src, f"<mutant {name}>", "exec"), ns)
+    return ns[name]
+
+
+def caught(fn, *args):
+    try:
+        fn(*args)
+    except (AssertionError, ValueError, FloatingPointError, IndexError, ZeroDivisionError):
+        return True
+    return False
+
+
+ATTEND_MUTANTS = [
+    ("dropped scale", "s = scale * (q @ k.T)", "s = (q @ k.T)"),
+    ("softmax over the query axis", "mx = s.max(axis=1, keepdims=True)", "mx = s.max(axis=0, keepdims=True)"),
+    ("normaliser summed over queries", "z = e.sum(axis=1)", "z = e.sum(axis=0)"),
+    ("L without the max", "l = mx[:, 0] + np.log(z)", "l = np.log(z)"),
+    ("wrong sign in the exponent", "e = np.exp(s - mx)", "e = np.exp(mx - s)"),
+    ("unnormalised output", "a = (e @ v) / z[:, None]", "a = (e @ v)"),
+]
+
+MERGE_MUTANTS = [
+    ("weights swapped", "a = (w_out[..., None] * a_out + w_in[..., None] * a_in)",
+     "a = (w_in[..., None] * a_out + w_out[..., None] * a_in)"),
+    ("L_full drops the log term", "l = np.where(empty, -np.inf, m_safe + np.log(den_safe))",
+     "l = np.where(empty, -np.inf, m_safe)"),
+    ("denominator drops a term", "den = w_out + w_in", "den = w_out + 0 * w_in + (w_in > 2)"),
+    ("min instead of max", "m = np.maximum(l_out, l_in)", "m = np.minimum(l_out, l_in)"),
+    ("both-empty merge gives L = 0", "l = np.where(empty, -np.inf, m_safe + np.log(den_safe))",
+     "l = np.where(empty, 0.0, m_safe + np.log(den_safe))"),
+]
+
+DECIDE_MUTANTS = [
+    ("tau: <= instead of <", "reuse &= (m < int(tau))[:, None]", "reuse &= (m <= int(tau))[:, None]"),
+    ("gamma: >= instead of >", "reuse &= np.asarray(cos) > np.float64(gamma)",
+     "reuse &= np.asarray(cos) >= np.float64(gamma)"),
+    ("gates OR-ed", "reuse &= np.asarray(cos) > np.float64(gamma)",
+     "reuse |= np.asarray(cos) > np.float64(gamma)"),
+    ("invalid cache ignored", "return ~(reuse & valid)", "return ~reuse"),
+    ("force reuse ignored", "if flags & FORCE_REUSE:", "if flags & 0:"),
+]
+
+COSINE_MUTANTS = [
+    ("no square root", "den = np.sqrt(np.dot(x, x) * np.dot(y, y))", "den = np.dot(x, x) * np.dot(y, y)"),
+    ("cache addressed by packed row", "y = q_ref[crow[r0:r1], h].reshape(-1)", "y = q_ref[r0:r1, h].reshape(-1)"),
+]
+
+PROBLEM_MUTANTS = [
+    ("GQA mapping h % H_kv", "hs = [h for h in head_list if h // g == hk]",
+     "hs = [h for h in head_list if h % Hk == hk]"),
+    ("keys of every sequence", "k0, k1 = _key_range(problem, which, b)",
+     "k0, k1 = 0, int(k_bits.shape[0])"),
+]
+
+
+@pytest.mark.parametrize("label,old,new", ATTEND_MUTANTS, ids=[m[0] for m in ATTEND_MUTANTS])
+def test_attend_mutants_caught(label, old, new):
+    bad = mutate(attention, "attend", old, new)
+    assert (caught(pins.check_golden_attend, bad) or caught(pins.check_brute_force, bad)
+            or caught(pins.check_closed_forms, bad)), label
+
+
+@pytest.mark.parametrize("label,old,new", MERGE_MUTANTS, ids=[m[0] for m in MERGE_MUTANTS])
+def test_merge_mutants_caught(label, old, new):
+    bad = mutate(attention, "merge", old, new)
+    assert (caught(pins.check_golden_merge, bad)
+            or caught(pins.check_fresh_cache_identity, attention.attend, bad)
+            or caught(pins.check_merge_order_independent, attention.attend, bad)), label
+
+
+@pytest.mark.parametrize("label,old,new", DECIDE_MUTANTS, ids=[m[0] for m in DECIDE_MUTANTS])
+def test_decide_mutants_caught(label, old, new):
+    bad = mutate(policy, "decide", old, new)
+    assert caught(pins.check_golden_gates, bad), label
+
+
+@pytest.mark.parametrize("label,old,new", COSINE_MUTANTS, ids=[m[0] for m in COSINE_MUTANTS])
+def test_cosine_mutants_caught(label, old, new):
+    bad = mutate(policy, "head_cosine", old, new)
+    assert caught(pins.check_cosine, bad), label
+
+
+@pytest.mark.parametrize("label,old,new", PROBLEM_MUTANTS, ids=[m[0] for m in PROBLEM_MUTANTS])
+def test_problem_mutants_caught(label, old, new):
+    bad = mutate(attention, "attend_problem", old, new)
+    assert caught(pins.check_problem_vs_brute, bad, attention.merge), label
+
+
+def test_unmutated_oracle_passes_every_pin():
+    pins.check_golden_attend(attention.attend)
+    pins.check_brute_force(attention.attend)
+    pins.check_closed_forms(attention.attend)
+    pins.check_golden_merge(attention.merge)
+    pins.check_fresh_cache_identity(attention.attend, attention.merge)
+    pins.check_merge_order_independent(attention.attend, attention.merge)
+    pins.check_golden_gates(policy.decide)
+    pins.check_cosine(policy.head_cosine)
+    pins.check_problem_vs_brute(attention.attend_problem, attention.merge)
