@@ -1,0 +1,512 @@
+// Host side of the C ABI declared in include/flashblock.h: argument checks,
+// launch planning, the TMA descriptor cache and the kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+
+#include "fb_kernels.cuh"
+#include "flashblock.h"
+
+namespace {
+
+thread_local std::string t_err = "no error";
+
+fb_status fail(fb_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return s;
+}
+
+fb_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FB_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ validation
+
+fb_status check_problem(const fb_problem* p) {
+  if (!p) return fail(FB_ERR_INVALID_ARG, "problem is NULL");
+  if (p->num_seqs < 0) return fail(FB_ERR_INVALID_ARG, "num_seqs < 0");
+  if (p->num_heads_q <= 0 || p->num_heads_kv <= 0) return fail(FB_ERR_INVALID_ARG, "head counts must be > 0");
+  if (p->num_heads_q % p->num_heads_kv != 0)
+    return fail(FB_ERR_UNSUPPORTED, "num_heads_q (%d) is not a multiple of num_heads_kv (%d)", p->num_heads_q,
+                p->num_heads_kv);
+  if (p->num_heads_q / p->num_heads_kv > fb::kMaxGroup)
+    return fail(FB_ERR_UNSUPPORTED, "query heads per kv head > %d", fb::kMaxGroup);
+  if (p->head_dim != 64 && p->head_dim != 128) return fail(FB_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", p->head_dim);
+  if (!(p->softmax_scale > 0.f) || !std::isfinite(p->softmax_scale))
+    return fail(FB_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (p->total_q < 0 || p->total_kv_out < 0 || p->total_kv_in < 0 || p->max_q < 0 || p->max_kv_out < 0 ||
+      p->max_kv_in < 0)
+    return fail(FB_ERR_INVALID_ARG, "negative size");
+  if (p->max_q > p->total_q || p->max_kv_out > p->total_kv_out || p->max_kv_in > p->total_kv_in)
+    return fail(FB_ERR_INVALID_ARG, "a per-sequence maximum exceeds its total");
+  if (p->max_q > p->max_kv_in) return fail(FB_ERR_INVALID_ARG, "max_q exceeds max_kv_in (rows are block positions)");
+  if (p->out_splits < 0) return fail(FB_ERR_INVALID_ARG, "out_splits < 0");
+  if (p->num_seqs > 0 && (!p->cu_seqlens_q || !p->cu_seqlens_kv_out || !p->cu_seqlens_kv_in))
+    return fail(FB_ERR_INVALID_ARG, "cu_seqlens arrays must not be NULL");
+  return FB_OK;
+}
+
+fb_status check_ptr(const void* ptr, const char* name, bool needed) {
+  if (!needed) return FB_OK;
+  if (!ptr) return fail(FB_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(ptr)) return fail(FB_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return FB_OK;
+}
+
+#define FB_TRY(x)                     \
+  do {                                \
+    fb_status _s = (x);               \
+    if (_s != FB_OK) return _s;       \
+  } while (0)
+
+// ------------------------------------------------------------------ planning
+
+struct Plan {
+  int d = 0, g = 0, wm = 0, wn = 0, tr = 0, tiles = 0, n_groups = 0, splits = 1, kps = fb::kBN, slots = 2;
+  size_t off_group_ctr = 0, off_grid_ctr = 0, off_cos = 0, off_part_a = 0, off_part_l = 0, bytes = 0;
+};
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int smem_bytes(int d, int wm);  // defined with the kernel table
+
+Plan make_plan(const fb_problem* p, int num_sms) {
+  Plan pl;
+  pl.d = p->head_dim;
+  pl.g = p->num_heads_q / p->num_heads_kv;
+  const long rows = static_cast<long>(pl.g) * p->max_q;
+  pl.wm = rows <= 16 ? 1 : rows <= 32 ? 2 : rows <= 64 ? 4 : 8;
+  pl.wn = pl.wm <= 2 ? 4 : pl.wm == 4 ? 2 : 1;
+  pl.tr = 16 * pl.wm;
+  pl.tiles = std::max<long>(1, (rows + pl.tr - 1) / pl.tr);
+  pl.n_groups = p->num_seqs * p->num_heads_kv * pl.tiles;
+  const int chunks = std::max(1, (p->max_kv_out + fb::kBN - 1) / fb::kBN);
+  int splits = p->out_splits;
+  if (splits <= 0) {
+    // Minimise waves x (chunks per split + a fixed per-CTA cost of ~2 chunks: the
+    // Q tile, the partial write and the merge) over the CTA slots of the GPU; on
+    // ties prefer more CTAs (more loads in flight).
+    const int per_sm = std::max(1, std::min(2, 200 * 1024 / std::max(1, smem_bytes(pl.d, pl.wm))));
+    const long slots = static_cast<long>(num_sms) * per_sm;
+    long best = -1;
+    splits = 1;
+    const int max_s = std::min(chunks, 64);
+    for (int s = 1; s <= max_s; ++s) {
+      const int cps = (chunks + s - 1) / s;
+      const int s_eff = (chunks + cps - 1) / cps;
+      const long ctas = static_cast<long>(pl.n_groups) * s_eff;
+      const long waves = std::max(1L, (ctas + slots - 1) / slots);
+      const long cost = waves * (cps + 2);
+      if (best < 0 || cost <= best) {
+        best = cost;
+        splits = s_eff;
+      }
+    }
+  }
+  splits = std::max(1, std::min(splits, chunks));
+  const int cps = (chunks + splits - 1) / splits;
+  pl.kps = cps * fb::kBN;
+  pl.splits = (chunks + cps - 1) / cps;
+  pl.slots = pl.splits + 1;
+  // workspace layout
+  size_t off = 0;
+  pl.off_group_ctr = off;
+  off = align_up(off + sizeof(int) * std::max(1, pl.n_groups), 256);
+  pl.off_grid_ctr = off;
+  off = align_up(off + sizeof(int), 256);
+  pl.off_cos = off;
+  off = align_up(off + sizeof(float) * std::max(1, p->num_seqs * p->num_heads_q), 256);
+  pl.off_part_a = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(pl.n_groups) * pl.slots * pl.tr * pl.d, 256);
+  pl.off_part_l = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(pl.n_groups) * pl.slots * pl.tr, 256);
+  pl.bytes = off;
+  return pl;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_map_mu;
+std::unordered_map<std::string, CUtensorMap> g_maps;
+EncodeTiledFn g_encode = nullptr;
+
+fb_status get_encode(EncodeTiledFn* fn) {
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (!g_encode) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f)
+      return fail(FB_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    g_encode = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  *fn = g_encode;
+  return FB_OK;
+}
+
+// Map of a THD bf16 buffer [tokens, hkv, d] viewed as 2-D {hkv*d, tokens}; the box
+// is 64 columns (128 bytes, the swizzle span) by kBN token rows.
+fb_status kv_map(const void* ptr, int tokens, int hkv, int d, CUtensorMap* out) {
+  std::memset(out, 0, sizeof(*out));
+  if (tokens <= 0) return FB_OK;  // never read: every key range is empty
+  int dev = 0;
+  cudaGetDevice(&dev);
+  char key[96];
+  snprintf(key, sizeof(key), "%d:%p:%d:%d:%d", dev, ptr, tokens, hkv, d);
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return FB_OK;
+    }
+  }
+  EncodeTiledFn enc;
+  FB_TRY(get_encode(&enc));
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(hkv) * d, static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(hkv) * d * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(fb::kBN)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FB_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (g_maps.size() > 4096) g_maps.clear();
+  g_maps.emplace(key, *out);
+  return FB_OK;
+}
+
+// ------------------------------------------------------------------ kernel table
+
+template <int D, int WM>
+struct KernelFor {
+  static constexpr int WN = WM <= 2 ? 4 : (WM == 4 ? 2 : 1);
+  using C = fb::Cfg<D, WM, WN>;
+  static void* fn() { return reinterpret_cast<void*>(&fb::attn_kernel<D, WM, WN>); }
+};
+
+struct KernelInfo {
+  void* fn;
+  int threads;
+  int smem;
+};
+
+template <int D, int WM>
+KernelInfo info_of() {
+  using K = KernelFor<D, WM>;
+  return {K::fn(), K::C::kThreads, K::C::kSmem};
+}
+
+KernelInfo kernel_info(int d, int wm) {
+  if (d == 64) {
+    switch (wm) {
+      case 1: return info_of<64, 1>();
+      case 2: return info_of<64, 2>();
+      case 4: return info_of<64, 4>();
+      default: return info_of<64, 8>();
+    }
+  }
+  switch (wm) {
+    case 1: return info_of<128, 1>();
+    case 2: return info_of<128, 2>();
+    case 4: return info_of<128, 4>();
+    default: return info_of<128, 8>();
+  }
+}
+
+int smem_bytes(int d, int wm) { return kernel_info(d, wm).smem; }
+
+fb_status launch_attn(const Plan& pl, fb::Params& prm, int n_ctas, cudaStream_t stream) {
+  if (n_ctas <= 0) return FB_OK;
+  KernelInfo ki = kernel_info(pl.d, pl.wm);
+  static std::mutex mu;
+  static bool attr_done[2][9] = {};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    bool& done = attr_done[pl.d == 128][pl.wm];
+    if (!done) {
+      cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, ki.smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      done = true;
+    }
+  }
+  void* args[] = {&prm};
+  cudaError_t e = cudaLaunchKernel(ki.fn, dim3(n_ctas), dim3(ki.threads), args, ki.smem, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  return FB_OK;
+}
+
+void fill_problem(const fb_problem* p, const Plan& pl, fb::Params& prm) {
+  prm.num_seqs = p->num_seqs;
+  prm.hq = p->num_heads_q;
+  prm.hkv = p->num_heads_kv;
+  prm.g = pl.g;
+  prm.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+  prm.cu_q = p->cu_seqlens_q;
+  prm.q_rows = p->q_rows;
+  prm.cu_out = p->cu_seqlens_kv_out;
+  prm.cu_in = p->cu_seqlens_kv_in;
+  prm.total_q = p->total_q;
+  prm.total_out = p->total_kv_out;
+  prm.total_in = p->total_kv_in;
+  prm.tr = pl.tr;
+  prm.tiles = pl.tiles;
+  prm.n_groups = pl.n_groups;
+  prm.splits = pl.splits;
+  prm.kps = pl.kps;
+  prm.slots = pl.slots;
+}
+
+void fill_workspace(const Plan& pl, void* ws, fb::Params& prm) {
+  char* base = static_cast<char*>(ws);
+  prm.group_ctr = reinterpret_cast<int*>(base + pl.off_group_ctr);
+  prm.grid_ctr = reinterpret_cast<int*>(base + pl.off_grid_ctr);
+  prm.cos = reinterpret_cast<const float*>(base + pl.off_cos);
+  prm.part_a = reinterpret_cast<float*>(base + pl.off_part_a);
+  prm.part_l = reinterpret_cast<float*>(base + pl.off_part_l);
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+
+extern "C" {
+
+const char* fb_last_error(void) { return t_err.c_str(); }
+
+int32_t fb_version(void) { return 100; }
+
+fb_status fb_workspace_size(const fb_problem* problem, size_t* bytes) {
+  FB_TRY(check_problem(problem));
+  if (!bytes) return fail(FB_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = make_plan(problem, device_sms()).bytes;
+  return FB_OK;
+}
+
+fb_status fb_workspace_init(void* workspace, size_t bytes, fb_stream_t stream) {
+  if (!workspace && bytes) return fail(FB_ERR_INVALID_ARG, "workspace is NULL");
+  if (!bytes) return FB_OK;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, bytes, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+  return FB_OK;
+}
+
+fb_status fb_out_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16* k_out, const fb_bf16* v_out,
+                      const uint8_t* head_mask, float* a_out, float* l_out, void* workspace, size_t workspace_bytes,
+                      fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  const bool rows = problem->total_q > 0;
+  FB_TRY(check_ptr(q, "q", rows));
+  FB_TRY(check_ptr(k_out, "k_out", problem->total_kv_out > 0));
+  FB_TRY(check_ptr(v_out, "v_out", problem->total_kv_out > 0));
+  FB_TRY(check_ptr(a_out, "a_out", rows));
+  if (rows && !l_out) return fail(FB_ERR_INVALID_ARG, "l_out is NULL");
+  if (problem->num_seqs == 0 || !rows) return FB_OK;
+  const Plan pl = make_plan(problem, device_sms());
+  if (!workspace || workspace_bytes < pl.bytes)
+    return fail(FB_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, pl.bytes);
+  fb::Params prm;
+  std::memset(&prm, 0, sizeof(prm));
+  fill_problem(problem, pl, prm);
+  fill_workspace(pl, workspace, prm);
+  FB_TRY(kv_map(k_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, &prm.tm_k_out));
+  FB_TRY(kv_map(v_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, &prm.tm_v_out));
+  prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  prm.do_out = 1;
+  prm.head_mask = head_mask;
+  prm.cache_a = a_out;
+  prm.cache_l = l_out;
+  prm.n_in_ctas = 0;
+  return launch_attn(pl, prm, pl.n_groups * pl.splits, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16* k_in, const fb_bf16* v_in,
+                     float* a_in, float* l_in, fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  const bool rows = problem->total_q > 0;
+  FB_TRY(check_ptr(q, "q", rows));
+  FB_TRY(check_ptr(k_in, "k_in", problem->total_kv_in > 0));
+  FB_TRY(check_ptr(v_in, "v_in", problem->total_kv_in > 0));
+  FB_TRY(check_ptr(a_in, "a_in", rows));
+  if (rows && !l_in) return fail(FB_ERR_INVALID_ARG, "l_in is NULL");
+  if (problem->num_seqs == 0 || !rows) return FB_OK;
+  const Plan pl = make_plan(problem, device_sms());
+  fb::Params prm;
+  std::memset(&prm, 0, sizeof(prm));
+  fill_problem(problem, pl, prm);
+  FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, &prm.tm_k_in));
+  FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, &prm.tm_v_in));
+  prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  prm.do_in = 1;
+  prm.a_in = a_in;
+  prm.l_in = l_in;
+  prm.n_in_ctas = pl.n_groups;
+  return launch_attn(pl, prm, pl.n_groups, reinterpret_cast<cudaStream_t>(stream));
+}
+
+fb_status fb_merge(int64_t n, int32_t d, const float* a_out, const float* l_out, const float* a_in,
+                   const float* l_in, float* a_full_f32, fb_bf16* a_full_bf16, float* l_full, fb_stream_t stream) {
+  if (n < 0 || d <= 0) return fail(FB_ERR_INVALID_ARG, "n must be >= 0 and d > 0");
+  if (n == 0) return FB_OK;
+  if (!a_out || !l_out || !a_in || !l_in) return fail(FB_ERR_INVALID_ARG, "merge inputs must not be NULL");
+  if (!a_full_f32 && !a_full_bf16) return fail(FB_ERR_INVALID_ARG, "no output for A_full");
+  fb::MergeParams mp{n, d, a_out, l_out, a_in, l_in, a_full_f32, reinterpret_cast<__nv_bfloat16*>(a_full_bf16),
+                     l_full};
+  const int64_t total = n * static_cast<int64_t>(d);
+  const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));
+  fb::merge_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(mp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
+  return FB_OK;
+}
+
+fb_status fb_head_similarity(const fb_problem* problem, const fb_bf16* q, const fb_bf16* q_ref, float* cos_out,
+                             fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  FB_TRY(check_ptr(q, "q", problem->total_q > 0));
+  FB_TRY(check_ptr(q_ref, "q_ref", problem->total_kv_in > 0));
+  if (!cos_out && problem->num_seqs > 0) return fail(FB_ERR_INVALID_ARG, "cos_out is NULL");
+  if (problem->num_seqs == 0) return FB_OK;
+  fb::SimParams sp{problem->num_heads_q, problem->head_dim, problem->total_q, problem->total_kv_in,
+                   problem->cu_seqlens_q, problem->q_rows,
+                   problem->cu_seqlens_kv_in, reinterpret_cast<const __nv_bfloat16*>(q),
+                   reinterpret_cast<const __nv_bfloat16*>(q_ref), cos_out};
+  fb::similarity_kernel<<<problem->num_seqs * problem->num_heads_q, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      sp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "similarity kernel launch");
+  return FB_OK;
+}
+
+fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_cache* cache, const fb_bf16* q,
+                  const fb_bf16* k_in, const fb_bf16* v_in, const fb_bf16* k_out, const fb_bf16* v_out,
+                  const int32_t* n_updated, const uint8_t* head_reuse_in, fb_bf16* a_full, float* l_full,
+                  uint8_t* decision_out, void* workspace, size_t workspace_bytes, fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  if (!params) return fail(FB_ERR_INVALID_ARG, "params is NULL");
+  if (!cache) return fail(FB_ERR_INVALID_ARG, "cache is NULL");
+  const unsigned flags = params->flags;
+  if (flags & ~15u) return fail(FB_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags & ~15u);
+  if ((flags & FB_FORCE_RECOMPUTE) && (flags & FB_FORCE_REUSE))
+    return fail(FB_ERR_INVALID_ARG, "FB_FORCE_RECOMPUTE and FB_FORCE_REUSE are exclusive");
+  const bool rows = problem->total_q > 0;
+  const bool uses_gates = !(flags & (FB_FORCE_RECOMPUTE | FB_FORCE_REUSE)) && !head_reuse_in;
+  const bool head_gate = uses_gates && (flags & FB_GATE_HEAD);
+  if (uses_gates && (flags & FB_GATE_TAU) && !n_updated)
+    return fail(FB_ERR_INVALID_ARG, "FB_GATE_TAU needs n_updated");
+  if (head_gate && !cache->q_ref) return fail(FB_ERR_INVALID_ARG, "FB_GATE_HEAD needs cache->q_ref");
+  if (head_gate && !(params->gamma == params->gamma)) return fail(FB_ERR_INVALID_ARG, "gamma is NaN");
+  FB_TRY(check_ptr(q, "q", rows));
+  FB_TRY(check_ptr(k_in, "k_in", problem->total_kv_in > 0));
+  FB_TRY(check_ptr(v_in, "v_in", problem->total_kv_in > 0));
+  FB_TRY(check_ptr(k_out, "k_out", problem->total_kv_out > 0));
+  FB_TRY(check_ptr(v_out, "v_out", problem->total_kv_out > 0));
+  FB_TRY(check_ptr(a_full, "a_full", rows));
+  FB_TRY(check_ptr(cache->a_out, "cache->a_out", problem->total_kv_in > 0));
+  if (problem->total_kv_in > 0 && !cache->l_out) return fail(FB_ERR_INVALID_ARG, "cache->l_out is NULL");
+  if (problem->num_seqs > 0 && !cache->valid) return fail(FB_ERR_INVALID_ARG, "cache->valid is NULL");
+  if (cache->q_ref) FB_TRY(check_ptr(cache->q_ref, "cache->q_ref", true));
+  if (problem->num_seqs == 0) return FB_OK;
+  const Plan pl = make_plan(problem, device_sms());
+  if (!workspace || workspace_bytes < pl.bytes)
+    return fail(FB_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, pl.bytes);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  fb::Params prm;
+  std::memset(&prm, 0, sizeof(prm));
+  fill_problem(problem, pl, prm);
+  fill_workspace(pl, workspace, prm);
+  FB_TRY(kv_map(k_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, &prm.tm_k_out));
+  FB_TRY(kv_map(v_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, &prm.tm_v_out));
+  FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, &prm.tm_k_in));
+  FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, &prm.tm_v_in));
+
+  if (head_gate && rows) {
+    float* cos_ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_cos);
+    FB_TRY(fb_head_similarity(problem, q, cache->q_ref, cos_ws, stream));
+  }
+  prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  prm.do_out = 1;
+  prm.do_in = 1;
+  prm.fused = 1;
+  prm.update_state = 1;
+  prm.flags = flags;
+  prm.tau = params->tau;
+  prm.gamma = params->gamma;
+  prm.n_updated = n_updated;
+  prm.head_reuse_in = head_reuse_in;
+  prm.cache_a = cache->a_out;
+  prm.cache_l = cache->l_out;
+  prm.valid = cache->valid;
+  prm.q_ref = reinterpret_cast<__nv_bfloat16*>(cache->q_ref);
+  prm.a_full = reinterpret_cast<__nv_bfloat16*>(a_full);
+  prm.l_full = l_full;
+  prm.decision_out = decision_out;
+  prm.n_in_ctas = pl.n_groups;
+  return launch_attn(pl, prm, pl.n_groups * (1 + pl.splits), st);
+}
+
+fb_status fb_cache_invalidate(const fb_problem* problem, const fb_cache* cache, fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  if (!cache || (!cache->valid && problem->num_seqs > 0)) return fail(FB_ERR_INVALID_ARG, "cache->valid is NULL");
+  const size_t n = static_cast<size_t>(problem->num_seqs) * problem->num_heads_q;
+  if (!n) return FB_OK;
+  cudaError_t e = cudaMemsetAsync(cache->valid, 0, n, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(valid)");
+  return FB_OK;
+}
+
+fb_status fb_release_cache(void) {
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  g_maps.clear();
+  return FB_OK;
+}
+
+fb_status fb_device_status(int32_t* code, fb_stream_t stream) {
+  if (!code) return fail(FB_ERR_INVALID_ARG, "code is NULL");
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, fb::g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(fb::g_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  *code = v;
+  return FB_OK;
+}
+
+}  // extern "C"

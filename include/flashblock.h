@@ -1,0 +1,213 @@
+/*
+ * flashblock.h -- C ABI of the FlashBlock denoise-step attention library (B200, sm_100a).
+ *
+ * What the library computes (FlashBlock, gist.science/es/paper/2602.05305,
+ * "Mecanismo Central"): the queries of the active block attend to two key sets,
+ * J_out (tokens outside the block: the cached prefix) and J_in (the block's own
+ * tokens, bidirectional).  Each set gives a partial (A, L): A is softmax
+ * attention over the set and L = log Z its natural-log normaliser.  The
+ * out-of-block partial (A_out, L_out) is cached and reused on later steps; the
+ * full output is the log-space composition
+ *     A_full = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (e^{L_out-m} + e^{L_in-m}),
+ *     m = max(L_out, L_in),
+ * with L_full = m + ln(e^{L_out-m} + e^{L_in-m}).
+ * Reuse is decided per (sequence, q-head) by the gates of FlashBlock's
+ * "Estrategias de Reutilizacion Adaptativa" (threshold tau on the updated-token
+ * count; per-head similarity gamma) and only active query rows are computed
+ * (SureLock, gist.science/es/paper/2602.06412, "Mecanismo de Funcionamiento":
+ * locked rows compute no query but their K/V are still attended).  Several
+ * requests or branches are packed into one call with cu_seqlens offsets
+ * (BlockBatch, gist.science/fr/paper/2605.29233, "Optimisation Systeme").
+ *
+ * Conventions
+ *  - Layout "THD": [tokens, heads, head_dim], head_dim contiguous, row-major.
+ *  - bf16 tensors are passed as raw 16-bit patterns (fb_bf16).
+ *  - Pointers marked (device) must be CUDA device memory of the current device;
+ *    pointers marked (host) are host memory.  The caller owns every buffer; no
+ *    call allocates device memory.  Every bf16/fp32 tensor must be 16-byte aligned.
+ *  - Calls validate on the host and then enqueue on `stream` without
+ *    synchronising (except fb_device_status).  They never abort or exit; on
+ *    failure they return a non-zero fb_status and fb_last_error() describes it.
+ *    Argument checks happen before any CUDA call, so they also work on a
+ *    machine without a GPU.
+ *  - softmax scale: scores are s = softmax_scale * q.k (usually 1/sqrt(d)).
+ *  - Grouped heads: q-head h reads kv-head h / (num_heads_q / num_heads_kv).
+ *  - Empty key set: A = 0, L = -inf.  Merging with an empty side returns the
+ *    other side; two empty sides give A = 0, L = -inf.
+ *  - A kernel that waits on an asynchronous copy gives up after about two
+ *    seconds, records FB_ERR_TIMEOUT in a device status word and returns;
+ *    fb_device_status() reads and clears it.  After a timeout the workspace
+ *    must be re-initialised with fb_workspace_init().
+ */
+#ifndef FLASHBLOCK_H
+#define FLASHBLOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t fb_bf16;                /* bf16 bit pattern */
+typedef struct CUstream_st* fb_stream_t; /* same type as cudaStream_t; NULL = default stream */
+
+typedef enum fb_status {
+  FB_OK = 0,
+  FB_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned buffer, bad offsets */
+  FB_ERR_UNSUPPORTED = 2, /* head_dim not 64/128, num_heads_q % num_heads_kv != 0, group > 32 */
+  FB_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (message has the CUDA error) */
+  FB_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out (see fb_device_status) */
+} fb_status;
+
+/* Gate flags of fb_params.flags. */
+#define FB_GATE_TAU 1u        /* reuse only if n_updated[b] < tau (strict)               */
+#define FB_GATE_HEAD 2u       /* reuse head h only if cos(Q_bh, q_ref_bh) > gamma (strict) */
+#define FB_FORCE_RECOMPUTE 4u /* recompute every head (dense step)                        */
+#define FB_FORCE_REUSE 8u     /* reuse every head whose cache is valid                    */
+
+/*
+ * One step's problem.  Index arrays are int32 device arrays; the scalar bounds
+ * are host values and must be exact totals / upper bounds of those arrays.
+ *   cu_seqlens_q      [num_seqs+1] offsets of each sequence's ACTIVE query rows in Q
+ *   q_rows            [total_q] block position (0..B_b-1) of each packed row, or
+ *                     NULL meaning row r of sequence b is block position r - cu_seqlens_q[b]
+ *   cu_seqlens_kv_out [num_seqs+1] offsets of each sequence's prefix (J_out) tokens
+ *   cu_seqlens_kv_in  [num_seqs+1] offsets of each sequence's block (J_in) tokens
+ * out_splits: number of key splits of the prefix pass; 0 lets the library choose.
+ */
+typedef struct fb_problem {
+  int32_t num_seqs, num_heads_q, num_heads_kv, head_dim;
+  float softmax_scale;
+  const int32_t* cu_seqlens_q;
+  const int32_t* q_rows;
+  const int32_t* cu_seqlens_kv_out;
+  const int32_t* cu_seqlens_kv_in;
+  int32_t total_q, total_kv_out, total_kv_in; /* host: Q / prefix / block token counts   */
+  int32_t max_q, max_kv_out, max_kv_in;       /* host: largest per-sequence count of each */
+  int32_t out_splits;
+} fb_problem;
+
+/*
+ * The FlashBlock cache (FlashBlock, "Mecanismo Central": A_out and L_out are kept
+ * from an earlier step and reused).  Rows are addressed by BLOCK POSITION, so a
+ * row keeps its entry while the active set shrinks:  cache row of packed row r of
+ * sequence b = cu_seqlens_kv_in[b] + q_rows[r].  All device memory, caller-owned.
+ *   a_out [total_kv_in, H_q, d] fp32;  l_out [total_kv_in, H_q] fp32
+ *   valid [num_seqs, H_q] uint8 (0 = empty: the head recomputes whatever the gates say)
+ *   q_ref [total_kv_in, H_q, d] bf16: the queries each head's entry was built with
+ *         (needed by FB_GATE_HEAD; may be NULL otherwise)
+ */
+typedef struct fb_cache {
+  float* a_out;
+  float* l_out;
+  uint8_t* valid;
+  fb_bf16* q_ref;
+} fb_cache;
+
+typedef struct fb_params {
+  int32_t tau;    /* threshold of FB_GATE_TAU */
+  float gamma;    /* threshold of FB_GATE_HEAD */
+  uint32_t flags; /* FB_GATE_* | FB_FORCE_* */
+} fb_params;
+
+/* Message of the last failing call on this thread (never NULL). */
+const char* fb_last_error(void);
+
+/* Library version (major*100 + minor). */
+int32_t fb_version(void);
+
+/*
+ * Bytes of workspace that fb_out_attn / fb_step / fb_head_similarity need for
+ * this problem (split partials, completion counters, similarity scores).  Pure
+ * host computation: plans for the current device's SM count, or for 148 SMs when
+ * no device is visible.
+ */
+fb_status fb_workspace_size(const fb_problem* problem, size_t* bytes);
+
+/* Zero a workspace (device) before its first use.  Calls leave it zeroed again. */
+fb_status fb_workspace_init(void* workspace, size_t bytes, fb_stream_t stream);
+
+/*
+ * Out-of-block partial (FlashBlock, "Mecanismo Central": A_out over J_out with
+ * L_out = log Z_out).  For every active row and every q-head h of sequence b
+ * with head_mask[b*H_q+h] != 0 (head_mask NULL = all heads), attends over all
+ * prefix tokens of b and writes (A_out, L_out) at the row's cache position:
+ *   a_out[(cu_seqlens_kv_in[b] + q_rows[r]) * H_q + h][0..d)  fp32
+ *   l_out[ same row * H_q + h ]                                fp32
+ * Heads with mask 0 are not touched.  q [total_q, H_q, d] bf16; k_out, v_out
+ * [total_kv_out, H_kv, d] bf16.  The prefix keys are split into key ranges whose
+ * partials are combined with the same log-space rule.
+ */
+fb_status fb_out_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16* k_out,
+                      const fb_bf16* v_out, const uint8_t* head_mask, float* a_out, float* l_out,
+                      void* workspace, size_t workspace_bytes, fb_stream_t stream);
+
+/*
+ * In-block partial (FlashBlock, "Mecanismo Central": A_in over J_in, the block's
+ * tokens, with no mask inside the block).  Locked tokens' K/V are part of J_in.
+ * Outputs in packed row order: a_in [total_q, H_q, d] fp32, l_in [total_q, H_q] fp32.
+ */
+fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16* k_in,
+                     const fb_bf16* v_in, float* a_in, float* l_in, fb_stream_t stream);
+
+/*
+ * Log-space merge of two partials (FlashBlock, "Mecanismo Central", the A_full
+ * equation), element-wise over n (row, head) entries of width d:
+ *   a_out, a_in [n, d] fp32;  l_out, l_in [n] fp32.
+ * Writes a_full_f32 [n, d] fp32 and/or a_full_bf16 [n, d] bf16 (either may be
+ * NULL, not both) and l_full [n] fp32 (may be NULL).  d any positive size.
+ */
+fb_status fb_merge(int64_t n, int32_t d, const float* a_out, const float* l_out, const float* a_in,
+                   const float* l_in, float* a_full_f32, fb_bf16* a_full_bf16, float* l_full,
+                   fb_stream_t stream);
+
+/*
+ * Per-head similarity of the FB_GATE_HEAD gate (FlashBlock, "Estrategias de
+ * Reutilizacion Adaptativa", per-head selection).  cos_out[b*H_q+h] = cosine
+ * between the active-row queries of (b, h), flattened rows x d, and q_ref at the
+ * same block positions.  fp32, fixed reduction order.  A zero denominator gives 0.
+ */
+fb_status fb_head_similarity(const fb_problem* problem, const fb_bf16* q, const fb_bf16* q_ref,
+                             float* cos_out, fb_stream_t stream);
+
+/*
+ * One denoise step of attention with the FlashBlock cache.
+ * Per (b, h): recompute = FORCE_RECOMPUTE or !valid[b,h] or (not FORCE_REUSE and
+ *   (head_reuse_in ? !head_reuse_in[b,h]
+ *                  : !((!GATE_TAU or n_updated[b] < tau) and (!GATE_HEAD or cos_bh > gamma)))).
+ * Heads that recompute get a fresh (A_out, L_out) over the prefix, stored in the
+ * cache with valid = 1 (and q_ref = the current queries when q_ref is not NULL);
+ * every head then attends over its block and merges with the cache:
+ *   a_full [total_q, H_q, d] bf16,  l_full [total_q, H_q] fp32 (may be NULL).
+ * n_updated [num_seqs] int32 (device; needed by FB_GATE_TAU).  head_reuse_in
+ * [num_seqs, H_q] uint8 (device, 1 = reuse) replaces the gates when not NULL.
+ * decision_out [num_seqs, H_q] uint8 (device, 1 = recomputed) may be NULL.
+ * The workspace must come from fb_workspace_size and be zeroed once
+ * (fb_workspace_init).  Calls on the same workspace must not overlap on the GPU.
+ */
+fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_cache* cache,
+                  const fb_bf16* q, const fb_bf16* k_in, const fb_bf16* v_in, const fb_bf16* k_out,
+                  const fb_bf16* v_out, const int32_t* n_updated, const uint8_t* head_reuse_in,
+                  fb_bf16* a_full, float* l_full, uint8_t* decision_out, void* workspace,
+                  size_t workspace_bytes, fb_stream_t stream);
+
+/* Mark every cache entry of the problem's sequences empty (valid = 0): a new
+ * block, a full refresh or a branch resync. */
+fb_status fb_cache_invalidate(const fb_problem* problem, const fb_cache* cache, fb_stream_t stream);
+
+/* Release the host-side tensor-map cache (descriptors of K/V buffers seen so far). */
+fb_status fb_release_cache(void);
+
+/* Synchronise `stream`, then read and clear the device status word:
+ * *code = FB_OK; FB_ERR_TIMEOUT if a bounded wait ran out since the last read;
+ * FB_ERR_INVALID_ARG if a kernel found an index array (cu_seqlens, q_rows) that
+ * disagrees with the host totals -- the affected work was skipped, not done out
+ * of bounds. */
+fb_status fb_device_status(int32_t* code, fb_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHBLOCK_H */

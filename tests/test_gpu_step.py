@@ -1,0 +1,84 @@
+"""fb_step (gates + out-of-block pass + in-block pass + merge) against the oracle
+applying the same reuse policy, step by step (needs a B200).
+
+Decisions are compared bit for bit; A_full within max-abs 2e-2 and mean-abs 1e-3,
+L_full within 1e-3 (bf16 inputs, fp32 accumulation)."""
+import numpy as np
+import pytest
+
+from cached_split_attention_b200 import workloads as W
+from gpu_util import assert_close, run_policy_gpu, torch_and_binding
+from oracle import policy
+
+pytestmark = pytest.mark.gpu
+
+
+def _compare(w, flags=None, out_splits=0, sample=None, head_reuse_in=None):
+    gpu, cache = run_policy_gpu(w, flags=flags, out_splits=out_splits, head_reuse_in=head_reuse_in)
+    ref = policy.run_policy(w, flags=flags, sample=sample, head_reuse_in=head_reuse_in)
+    for s, (g, r) in enumerate(zip(gpu, ref)):
+        assert np.array_equal(g["decision"], r.recompute), f"{w.name} step {s}: decisions differ"
+        if r.cos is not None and w.flags & W.GATE_HEAD:
+            assert np.all(np.abs(r.cos - w.gamma) > 1e-5), "a similarity sits within rounding of gamma"
+        assert_close(g["a_full"], r.a_full, g["l_full"], r.l_full, f"{w.name} step {s}")
+    return gpu, ref
+
+
+def test_tiny():
+    gpu, ref = _compare(W.tiny())
+    assert ref[0].recompute.all() and not any(r.recompute.any() for r in ref[1:])
+
+
+def test_tiny_sharp_forced_arms():
+    w = W.tiny(sharp=32.0)
+    _compare(w, flags=W.FORCE_RECOMPUTE)
+    _compare(w, flags=W.FORCE_REUSE)
+
+
+def test_tiny_multi_split():
+    _compare(W.tiny(), out_splits=3)
+
+
+def test_locking_monotone_gqa():
+    _compare(W.locking_tiny())
+
+
+def test_caller_head_mask():
+    w = W.locking_tiny(steps=3)
+    rng = np.random.default_rng(0)
+    masks = [None] + [rng.integers(0, 2, size=(w.problem.num_seqs, w.problem.num_heads_q)).astype(bool)
+                      for _ in range(2)]
+    _compare(w, head_reuse_in=masks)
+
+
+def test_dllm_layer_full_size():
+    """The 8B-dLLM layer workload at its full size, every row, all 32 steps."""
+    gpu, ref = _compare(W.dllm_layer())
+    dec = [bool(r.recompute.any()) for r in ref]
+    assert dec[0] and any(dec[1:]) and not all(dec[1:])
+
+
+def test_varlen_branches_full_size():
+    gpu, ref = _compare(W.varlen_branches())
+    per_branch = np.array([r.recompute[:, 0] for r in ref[1:]])
+    assert per_branch.any() and not per_branch.all()   # branches decide differently
+
+
+def test_long_context_gqa_reduced_both_arms():
+    w = W.long_context_gqa(steps=3, prefix=2048 + 37)
+    _compare(w, flags=W.FORCE_RECOMPUTE)
+    _compare(w, flags=W.FORCE_REUSE)
+
+
+def test_video_reduced_gamma_gate():
+    w = W.video(steps=4, block=256, prefix_blocks=2, heads=8)
+    gpu, ref = _compare(w)
+    assert any(r.recompute.any() and not r.recompute.all() for r in ref[1:])
+
+
+def test_determinism():
+    w = W.varlen_branches(steps=3, prefix=512)
+    a, _ = run_policy_gpu(w)
+    b, _ = run_policy_gpu(w)
+    for x, y in zip(a, b):
+        assert np.array_equal(x["a_full"], y["a_full"]) and np.array_equal(x["l_full"], y["l_full"])
