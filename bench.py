@@ -1,0 +1,529 @@
+"""Benchmark of the FlashBlock denoise-step attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload dllm_layer|long_context_gqa|varlen_branches|video|tiny]
+
+One bench step is one denoise episode of the workload's block (32 denoise steps
+for the 8B-dLLM layer: the cache is invalidated, step 0 recomputes, later steps
+follow the tau gate).  Every denoise step is one fb_step call (gates, out-of-block
+pass when recomputing, in-block pass, log-space merge) on resident inputs, timed
+with CUDA events on the launching stream; L2 is flushed (a 256 MiB read) before
+every denoise step and the flush is not timed.  `value` is the mean denoise-step
+latency in microseconds over the K timed episodes (max over ranks).
+
+`e2e` is the same metric through the public API with host buffers: each denoise
+step copies its block Q/K/V and update count from pinned host memory, calls
+fb_step and copies A_full and L_full back, all inside the timed region.
+
+`roofline` is the fused attention kernel on its recompute launches (the prefix
+pass: HBM-bound), with achieved = algorithmic bytes / launch time;
+`roofline_all_launches` aggregates every launch of the episode.
+
+`--impl reference` times the fp64 oracle (the plain CPU statement of the method)
+on the host cores on the same workload, one episode per step, rank 0 only.
+
+With torchrun (N > 1) every rank runs its own request (seed + rank) on its own
+GPU with no collective on the data path (weak scaling); ranks meet only at the
+barriers around the timed region and in the max-reduction of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from cached_split_attention_b200 import workloads as W  # noqa: E402
+
+METRIC = "denoise-step attention µs; effective KV TB/s vs ~8 TB/s HBM peak"
+WORKLOAD_DESC = {
+    "dllm_layer": "8B-dLLM layer: batch 1, bf16 MHA H=32, d=128, prefix 4096, block 32, 32 steps, "
+                  "1-4 redraws/step (Poisson mean 2), tau=4",
+    "long_context_gqa": "long context GQA: batch 8, H_q=32, H_kv=8, d=128, prefix 32768, block 64, "
+                        "16 steps, 50% rows locked, forced reuse after step 0",
+    "varlen_branches": "varlen branches: 6 branches B=4..128, prefix 2048 each, H=32, d=128, 8 steps, tau=4",
+    "video": "video-shaped: H=40, d=128, block 1560, prefix 9360, 10 steps, gamma=0.95",
+    "tiny": "tiny: H=4, d=64, prefix 256, block 32, 4 steps, tau=8",
+}
+
+
+# ---------------------------------------------------------------- algorithmic bytes
+
+def step_bytes(p, recompute_heads_frac: float) -> dict:
+    """Bytes the method must move in one denoise step (counted from the tensors):
+    Q rows + K/V of the block + A_full (bf16) and L_full, plus for heads that
+    recompute the prefix K/V and the cache write (A_out fp32 + L_out), and for
+    heads that reuse the cache read."""
+    H, Hk, d = p.num_heads_q, p.num_heads_kv, p.head_dim
+    q = p.total_q * H * d * 2
+    kv_in = p.total_kv_in * Hk * d * 2 * 2
+    out = p.total_q * H * (d * 2 + 4)
+    cache = p.total_q * H * (d * 4 + 4)
+    kv_out = p.total_kv_out * Hk * d * 2 * 2
+    f = recompute_heads_frac
+    return dict(total=q + kv_in + out + f * (kv_out + cache) + (1 - f) * cache,
+                kv_out=f * kv_out)
+
+
+def step_flops(p, recompute_heads_frac: float) -> float:
+    H, d = p.num_heads_q, p.head_dim
+    lens_q = np.diff(p.cu_seqlens_q).astype(np.float64)
+    lens_o = np.diff(p.cu_seqlens_kv_out).astype(np.float64)
+    lens_i = np.diff(p.cu_seqlens_kv_in).astype(np.float64)
+    return float(4 * H * d * (np.sum(lens_q * lens_i) + recompute_heads_frac * np.sum(lens_q * lens_o)))
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.period = period_s
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        mask = 0
+        for _, r in self.samples:
+            mask |= int(r)
+        reasons = [name for bit, name in self.REASONS.items() if mask & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank serves its own request: a different seed, same shapes."""
+    return base_seed + 7919 * rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def make_workload(name: str, seed: int):
+    fn = W.NAMED[name]
+    return fn(seed=seed)
+
+
+# ---------------------------------------------------------------- native arm
+
+class Episode:
+    """Device-resident inputs and buffers for one workload, run through fb_step."""
+
+    def __init__(self, w, device):
+        import torch
+        from cached_split_attention_b200 import binding as B
+        self.torch, self.B = torch, B
+        self.w = w
+        self.device = device
+        p = w.problem
+        self.dp = [B.DeviceProblem(st.problem, device) for st in w.steps]
+        self.cache = B.Cache(p, device, with_q_ref=bool(w.flags & W.GATE_HEAD))
+        self.k_out = B.bf16_tensor(w.k_out, device)
+        self.v_out = B.bf16_tensor(w.v_out, device)
+        self.q = [B.bf16_tensor(st.q, device) for st in w.steps]
+        self.k_in = [B.bf16_tensor(st.k_in, device) for st in w.steps]
+        self.v_in = [B.bf16_tensor(st.v_in, device) for st in w.steps]
+        self.n_upd = [torch.as_tensor(st.n_updated, dtype=torch.int32).to(device) for st in w.steps]
+        wsz = max(B.workspace_size(d) for d in self.dp)
+        self.ws = torch.empty(wsz, dtype=torch.uint8, device=device)
+        B.workspace_init(self.ws)
+        H, d = p.num_heads_q, p.head_dim
+        tq = max(st.problem.total_q for st in w.steps)
+        self.a_full = torch.empty((tq, H, d), dtype=torch.bfloat16, device=device)
+        self.l_full = torch.empty((tq, H), dtype=torch.float32, device=device)
+        self.dec = torch.empty((p.num_seqs, H), dtype=torch.uint8, device=device)
+        self.prm = B.params(w.tau, w.gamma, w.flags)
+        # pinned host copies for the end-to-end leg
+        self.h_q = [torch.from_numpy(st.q.view(np.int16)).pin_memory() for st in w.steps]
+        self.h_k = [torch.from_numpy(st.k_in.view(np.int16)).pin_memory() for st in w.steps]
+        self.h_v = [torch.from_numpy(st.v_in.view(np.int16)).pin_memory() for st in w.steps]
+        self.h_n = [torch.from_numpy(st.n_updated.astype(np.int32)).pin_memory() for st in w.steps]
+        self.d_q = torch.empty_like(self.q[0]).view(torch.int16)
+        self.d_k = torch.empty_like(self.k_in[0]).view(torch.int16)
+        self.d_v = torch.empty_like(self.v_in[0]).view(torch.int16)
+        self.d_n = torch.empty_like(self.n_upd[0])
+        self.h_a = torch.empty(self.a_full.shape, dtype=torch.bfloat16).pin_memory()
+        self.h_l = torch.empty(self.l_full.shape, dtype=torch.float32).pin_memory()
+        # L2 flush: read 256 MiB (about twice the L2) so that the next step starts
+        # with none of its data in L2 and no dirty lines to write back
+        self.flush_buf = torch.ones(64 << 20, dtype=torch.int32, device=device)
+        self.flush_out = torch.empty((), dtype=torch.int32, device=device)
+
+    def step(self, s, stream):
+        B = self.B
+        B.step(self.dp[s], self.prm, self.cache, self.q[s], self.k_in[s], self.v_in[s], self.k_out, self.v_out,
+               self.n_upd[s], self.a_full, self.ws, l_full=self.l_full, decision_out=self.dec, stream=stream)
+
+    def step_e2e(self, s, stream):
+        torch, B = self.torch, self.B
+        with torch.cuda.stream(stream):
+            self.d_q.copy_(self.h_q[s], non_blocking=True)
+            self.d_k.copy_(self.h_k[s], non_blocking=True)
+            self.d_v.copy_(self.h_v[s], non_blocking=True)
+            self.d_n.copy_(self.h_n[s], non_blocking=True)
+            B.step(self.dp[s], self.prm, self.cache, self.d_q.view(torch.bfloat16), self.d_k.view(torch.bfloat16),
+                   self.d_v.view(torch.bfloat16), self.k_out, self.v_out, self.d_n, self.a_full, self.ws,
+                   l_full=self.l_full, decision_out=self.dec, stream=stream)
+            tq = self.dp[s].host.total_q
+            self.h_a[:tq].copy_(self.a_full[:tq], non_blocking=True)
+            self.h_l[:tq].copy_(self.l_full[:tq], non_blocking=True)
+
+    def e2e_bytes(self, s):
+        st = self.w.steps[s]
+        tq = st.problem.total_q
+        H, d = self.w.problem.num_heads_q, self.w.problem.head_dim
+        return st.q.nbytes + st.k_in.nbytes + st.v_in.nbytes + st.n_updated.astype(np.int32).nbytes, \
+            tq * H * d * 2 + tq * H * 4
+
+    def flush(self, stream):
+        with self.torch.cuda.stream(stream):
+            self.torch.amax(self.flush_buf, dim=0, out=self.flush_out)
+
+    def run_episode(self, stream, events=None, e2e=False, flags=None):
+        """All denoise steps of the episode; events[s] = (start, end) per step."""
+        B = self.B
+        if flags is not None:
+            self.prm = B.params(self.w.tau, self.w.gamma, flags)
+        B.cache_invalidate(self.dp[0], self.cache, stream=stream)
+        decisions = []
+        for s in range(len(self.w.steps)):
+            self.flush(stream)
+            if events is not None:
+                events[s][0].record(stream)
+            if e2e:
+                self.step_e2e(s, stream)
+            else:
+                self.step(s, stream)
+            if events is not None:
+                events[s][1].record(stream)
+            decisions.append(None)
+        if flags is not None:
+            self.prm = B.params(self.w.tau, self.w.gamma, self.w.flags)
+        return decisions
+
+
+def native(args, world, rank, local):
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    base = {"tiny": 1000, "dllm_layer": 1001, "long_context_gqa": 1002, "varlen_branches": 1003,
+            "video": 1004}[args.workload]
+    w = make_workload(args.workload, shard_seed(base, rank))
+    ep = Episode(w, device)
+    stream = torch.cuda.current_stream(device)
+    S = len(w.steps)
+    p = w.problem
+
+    # The decisions of the episode (deterministic): run once to read them.
+    decisions = []
+    ep.B.cache_invalidate(ep.dp[0], ep.cache, stream=stream)
+    for s in range(S):
+        ep.step(s, stream)
+        decisions.append(ep.dec.cpu().numpy().astype(bool).copy())
+    rec_frac = [float(d.mean()) for d in decisions]
+
+    # warm-up episodes
+    for _ in range(args.warmup):
+        ep.run_episode(stream)
+    torch.cuda.synchronize()
+
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
+          for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        for k in range(args.steps):
+            ep.run_episode(stream, events=ev[k])
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = np.array([[ev[k][s][0].elapsed_time(ev[k][s][1]) for s in range(S)] for k in range(args.steps)])
+    episode_ms = float(step_ms.sum(axis=1).mean())
+    mean_step_us = float(step_ms.mean() * 1e3)
+
+    # end-to-end leg (host buffers, copies inside the timed region)
+    ev2 = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
+           for _ in range(args.steps)]
+    ep.run_episode(stream, e2e=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    for k in range(args.steps):
+        ep.run_episode(stream, events=ev2[k], e2e=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = np.array([[ev2[k][s][0].elapsed_time(ev2[k][s][1]) for s in range(S)] for k in range(args.steps)])
+    e2e_us = float(e2e_ms.mean() * 1e3)
+    h2d = sum(ep.e2e_bytes(s)[0] for s in range(S)) / S
+    d2h = sum(ep.e2e_bytes(s)[1] for s in range(S)) / S
+
+    # dense (forced recompute) and reuse (forced reuse) step latencies, L2 flushed
+    reps = max(3, min(args.steps, 20))
+    evd = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
+           for _ in range(reps)]
+    evr = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
+           for _ in range(reps)]
+    for k in range(reps):
+        ep.run_episode(stream, events=evd[k], flags=W.FORCE_RECOMPUTE)
+    for k in range(reps):
+        ep.run_episode(stream, events=evr[k], flags=W.FORCE_REUSE)
+    torch.cuda.synchronize()
+    dense_us = np.array([[evd[k][s][0].elapsed_time(evd[k][s][1]) * 1e3 for s in range(S)] for k in range(reps)])
+    reuse_us = np.array([[evr[k][s][0].elapsed_time(evr[k][s][1]) * 1e3 for s in range(1, S)] for k in range(reps)])
+
+    # roofline of the fused kernel: recompute launches of the timed episodes
+    rec_steps = [s for s in range(S) if rec_frac[s] > 0]
+    bytes_rec = sum(step_bytes(w.steps[s].problem, rec_frac[s])["total"] for s in rec_steps)
+    t_rec = step_ms[:, rec_steps].sum(axis=1).mean() * 1e-3 if rec_steps else float("nan")
+    bytes_all = sum(step_bytes(w.steps[s].problem, rec_frac[s])["total"] for s in range(S))
+    t_all = episode_ms * 1e-3
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    ach_rec = bytes_rec / t_rec / 1e9 if rec_steps else float("nan")
+    ach_all = bytes_all / t_all / 1e9
+    traffic = None
+    try:
+        prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        if prof.get("workload") == args.workload:
+            traffic = prof.get("dram_bytes_per_recompute_launch")
+    except Exception:
+        pass
+
+    value = max_over_ranks(mean_step_us, world, device)
+    e2e_v = max_over_ranks(e2e_us, world, device)
+    ms_step = max_over_ranks(episode_ms, world, device)
+    clocks = sampler.summary()
+    if rank != 0:
+        _teardown(world)
+        return
+
+    dense_b = step_bytes(p, 1.0)["total"]
+    reuse_b = step_bytes(p, 0.0)["total"]
+    dense_med = float(np.median(dense_us))
+    reuse_med = float(np.median(reuse_us))
+    out = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "us/denoise-step",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD_DESC[args.workload],
+            "bench_step": f"one denoise episode ({S} fb_step calls, cache invalidated at its start)",
+            "denoise_steps_per_episode": S,
+            "recompute_steps_per_episode": len(rec_steps),
+            "l2": "flushed before every denoise step (256 MiB read, untimed)",
+            "parallelism": f"replicas x{world} (one request per GPU, no collective)",
+            "seed": shard_seed(base, rank),
+        },
+        "throughput": {"denoise_steps_per_s_all_gpus": round(world * 1e6 / value, 1)},
+        "dense_step_us": {"median": round(dense_med, 3), "p10": round(float(np.percentile(dense_us, 10)), 3),
+                          "p90": round(float(np.percentile(dense_us, 90)), 3),
+                          "effective_tbps": round(dense_b / dense_med / 1e6, 3),
+                          "frac_of_hbm": round(dense_b / dense_med / 1e3 / hbm_peak, 4)},
+        "reuse_step_us": {"median": round(reuse_med, 3), "p10": round(float(np.percentile(reuse_us, 10)), 3),
+                          "p90": round(float(np.percentile(reuse_us, 90)), 3),
+                          "effective_tbps": round(reuse_b / reuse_med / 1e6, 3)},
+        "reuse_gain": {"predicted_bytes_ratio": round(dense_b / reuse_b, 2),
+                       "achieved_time_ratio": round(dense_med / reuse_med, 2)},
+        "roofline": {"bound": "hbm", "kernel": "attn_kernel (recompute launches: prefix pass + block pass + merge)",
+                     "achieved": round(ach_rec, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(ach_rec / hbm_peak, 4), "peak_source": peak_src, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": round(bytes_rec / max(1, len(rec_steps))),
+                     "launches": len(rec_steps) * args.steps},
+        "roofline_all_launches": {"achieved": round(ach_all, 1), "unit": "GB/s", "frac": round(ach_all / hbm_peak, 4),
+                                  "algorithmic_bytes_per_episode": round(bytes_all)},
+        "e2e": {"value": round(e2e_v, 3), "unit": "us/denoise-step", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(args.steps * S * (2 if w.flags & W.GATE_HEAD else 1)),
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, shard_seed(base, rank), budget_s=args.cpu_budget)
+    print(json.dumps(out), flush=True)
+    _teardown(world)
+
+
+def _teardown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- oracle on the host
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [os.cpu_count() or 1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(workload: str, seed: int, budget_s: float = 12.0) -> dict:
+    """The fp64 oracle (as it stands) on a bounded sample: whole episodes of the
+    same workload until about budget_s seconds have passed."""
+    from oracle import policy
+    w = make_workload(workload, seed)
+    S = len(w.steps)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        policy.run_policy(w)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(dt / (n * S) * 1e6, 1), "unit": "us/denoise-step", "cores": _oracle_threads(),
+            "kind": "oracle", "sample": f"{n} full episode(s) of {S} denoise steps, every row and head, fp64 numpy"}
+
+
+def reference(args, world, rank):
+    if rank != 0:
+        return
+    from oracle import policy
+    base = {"tiny": 1000, "dllm_layer": 1001, "long_context_gqa": 1002, "varlen_branches": 1003,
+            "video": 1004}[args.workload]
+    w = make_workload(args.workload, shard_seed(base, 0))
+    S = len(w.steps)
+    for _ in range(args.warmup):
+        policy.run_policy(w)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        policy.run_policy(w)
+    dt = time.perf_counter() - t0
+    us = dt / (args.steps * S) * 1e6
+    cores = _oracle_threads()
+    out = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(us, 1),
+        "unit": "us/denoise-step",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC[args.workload],
+                   "bench_step": f"one denoise episode ({S} steps) of the fp64 oracle on host cores"},
+        "cpu_baseline": {"value": round(us, 1), "unit": "us/denoise-step", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} full episode(s) of {S} denoise steps, every row and head"},
+        "e2e": {"value": round(us, 1), "unit": "us/denoise-step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_DESC), default="dllm_layer")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        reference(args, world, rank)
+    else:
+        native(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -77,8 +77,8 @@ fb_status check_ptr(const void* ptr, const char* name, bool needed) {
 // ------------------------------------------------------------------ planning
 
 struct Plan {
-  int d = 0, g = 0, wm = 0, wn = 0, tr = 0, tiles = 0, n_groups = 0, splits = 1, kps = fb::kBN, slots = 2;
-  size_t off_group_ctr = 0, off_grid_ctr = 0, off_cos = 0, off_part_a = 0, off_part_l = 0, bytes = 0;
+  int d = 0, g = 0, wm = 0, tr = 0, tiles = 0, n_groups = 0, splits = 1, threads = 0, smem = 0;
+  size_t off_grid_ctr = 0, off_cos = 0, off_in_a = 0, off_in_l = 0, bytes = 0;
 };
 
 int device_sms() {
@@ -96,58 +96,76 @@ int device_sms() {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-int smem_bytes(int d, int wm);  // defined with the kernel table
+// Tile shapes: WM row slabs of 16 rows x WN key shares = 8 warps per CTA (4 for
+// 16-row tiles), one CTA per SM; stage ring of 128 KB (96 KB for 128-row tiles).
+struct Shape {
+  void* fn;
+  int threads;
+  int smem;
+};
 
-Plan make_plan(const fb_problem* p, int num_sms) {
+template <int D, int WM>
+Shape shape_of() {
+  constexpr int WN = WM == 1 ? 4 : 8 / WM;
+  constexpr int ST = (D == 64 ? 2 : 1) * (WM == 8 ? 3 : 4);
+  using C = fb::Cfg<D, WM, WN, ST>;
+  return {reinterpret_cast<void*>(&fb::attn_kernel<D, WM, WN, ST>), C::kThreads, C::kSmem};
+}
+
+Shape shape_for(int d, int wm) {
+  if (d == 64) {
+    switch (wm) {
+      case 1: return shape_of<64, 1>();
+      case 2: return shape_of<64, 2>();
+      case 4: return shape_of<64, 4>();
+      default: return shape_of<64, 8>();
+    }
+  }
+  switch (wm) {
+    case 1: return shape_of<128, 1>();
+    case 2: return shape_of<128, 2>();
+    case 4: return shape_of<128, 4>();
+    default: return shape_of<128, 8>();
+  }
+}
+
+// in_only: fb_in_attn (no prefix pass, one CTA per group)
+Plan make_plan(const fb_problem* p, int num_sms, bool in_only) {
   Plan pl;
   pl.d = p->head_dim;
   pl.g = p->num_heads_q / p->num_heads_kv;
   const long rows = static_cast<long>(pl.g) * p->max_q;
   pl.wm = rows <= 16 ? 1 : rows <= 32 ? 2 : rows <= 64 ? 4 : 8;
-  pl.wn = pl.wm <= 2 ? 4 : pl.wm == 4 ? 2 : 1;
+  const Shape sh = shape_for(pl.d, pl.wm);
+  pl.threads = sh.threads;
+  pl.smem = sh.smem;
   pl.tr = 16 * pl.wm;
-  pl.tiles = std::max<long>(1, (rows + pl.tr - 1) / pl.tr);
+  pl.tiles = static_cast<int>(std::max<long>(1, (rows + pl.tr - 1) / pl.tr));
   pl.n_groups = p->num_seqs * p->num_heads_kv * pl.tiles;
   const int chunks = std::max(1, (p->max_kv_out + fb::kBN - 1) / fb::kBN);
-  int splits = p->out_splits;
-  if (splits <= 0) {
-    // Minimise waves x (chunks per split + a fixed per-CTA cost of ~2 chunks: the
-    // Q tile, the partial write and the merge) over the CTA slots of the GPU; on
-    // ties prefer more CTAs (more loads in flight).
-    const int per_sm = std::max(1, std::min(2, 200 * 1024 / std::max(1, smem_bytes(pl.d, pl.wm))));
-    const long slots = static_cast<long>(num_sms) * per_sm;
-    long best = -1;
-    splits = 1;
-    const int max_s = std::min(chunks, 64);
-    for (int s = 1; s <= max_s; ++s) {
-      const int cps = (chunks + s - 1) / s;
-      const int s_eff = (chunks + cps - 1) / cps;
-      const long ctas = static_cast<long>(pl.n_groups) * s_eff;
-      const long waves = std::max(1L, (ctas + slots - 1) / slots);
-      const long cost = waves * (cps + 2);
-      if (best < 0 || cost <= best) {
-        best = cost;
-        splits = s_eff;
-      }
+  int splits = 1;
+  if (!in_only) {
+    if (p->out_splits > 0) {
+      splits = p->out_splits;
+    } else {
+      // One wave: as many CTAs per group as the resident slots allow.
+      const int per_sm = std::max(1, std::min(233472 / (pl.smem + 1024), 2048 / pl.threads));
+      const long slots = static_cast<long>(num_sms) * per_sm;
+      splits = static_cast<int>(std::max(1L, slots / std::max(1, pl.n_groups)));
     }
+    splits = std::max(1, std::min({splits, fb::kMaxSplits, chunks}));
   }
-  splits = std::max(1, std::min(splits, chunks));
-  const int cps = (chunks + splits - 1) / splits;
-  pl.kps = cps * fb::kBN;
-  pl.splits = (chunks + cps - 1) / cps;
-  pl.slots = pl.splits + 1;
+  pl.splits = splits;
   // workspace layout
   size_t off = 0;
-  pl.off_group_ctr = off;
-  off = align_up(off + sizeof(int) * std::max(1, pl.n_groups), 256);
   pl.off_grid_ctr = off;
   off = align_up(off + sizeof(int), 256);
   pl.off_cos = off;
   off = align_up(off + sizeof(float) * std::max(1, p->num_seqs * p->num_heads_q), 256);
-  pl.off_part_a = off;
-  off = align_up(off + sizeof(float) * static_cast<size_t>(pl.n_groups) * pl.slots * pl.tr * pl.d, 256);
-  pl.off_part_l = off;
-  off = align_up(off + sizeof(float) * static_cast<size_t>(pl.n_groups) * pl.slots * pl.tr, 256);
+  pl.off_in_a = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(pl.n_groups) * pl.tr * pl.d, 256);
+  pl.off_in_l = off;
+  off = align_up(off + sizeof(float) * static_cast<size_t>(pl.n_groups) * pl.tr, 256);
   pl.bytes = off;
   return pl;
 }
@@ -209,62 +227,40 @@ fb_status kv_map(const void* ptr, int tokens, int hkv, int d, CUtensorMap* out) 
   return FB_OK;
 }
 
-// ------------------------------------------------------------------ kernel table
+// ------------------------------------------------------------------ launch
 
-template <int D, int WM>
-struct KernelFor {
-  static constexpr int WN = WM <= 2 ? 4 : (WM == 4 ? 2 : 1);
-  using C = fb::Cfg<D, WM, WN>;
-  static void* fn() { return reinterpret_cast<void*>(&fb::attn_kernel<D, WM, WN>); }
-};
-
-struct KernelInfo {
-  void* fn;
-  int threads;
-  int smem;
-};
-
-template <int D, int WM>
-KernelInfo info_of() {
-  using K = KernelFor<D, WM>;
-  return {K::fn(), K::C::kThreads, K::C::kSmem};
-}
-
-KernelInfo kernel_info(int d, int wm) {
-  if (d == 64) {
-    switch (wm) {
-      case 1: return info_of<64, 1>();
-      case 2: return info_of<64, 2>();
-      case 4: return info_of<64, 4>();
-      default: return info_of<64, 8>();
-    }
-  }
-  switch (wm) {
-    case 1: return info_of<128, 1>();
-    case 2: return info_of<128, 2>();
-    case 4: return info_of<128, 4>();
-    default: return info_of<128, 8>();
-  }
-}
-
-int smem_bytes(int d, int wm) { return kernel_info(d, wm).smem; }
-
-fb_status launch_attn(const Plan& pl, fb::Params& prm, int n_ctas, cudaStream_t stream) {
+fb_status launch_attn(const Plan& pl, fb::Params& prm, cudaStream_t stream) {
+  const int n_ctas = pl.n_groups * pl.splits;
   if (n_ctas <= 0) return FB_OK;
-  KernelInfo ki = kernel_info(pl.d, pl.wm);
+  void* fn = shape_for(pl.d, pl.wm).fn;
   static std::mutex mu;
   static bool attr_done[2][9] = {};
   {
     std::lock_guard<std::mutex> lk(mu);
     bool& done = attr_done[pl.d == 128][pl.wm];
     if (!done) {
-      cudaError_t e = cudaFuncSetAttribute(ki.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, ki.smem);
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       done = true;
     }
   }
+  prm.splits = pl.splits;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(n_ctas);
+  cfg.blockDim = dim3(pl.threads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (pl.splits > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
   void* args[] = {&prm};
-  cudaError_t e = cudaLaunchKernel(ki.fn, dim3(n_ctas), dim3(ki.threads), args, ki.smem, stream);
+  cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
   return FB_OK;
 }
@@ -282,21 +278,16 @@ void fill_problem(const fb_problem* p, const Plan& pl, fb::Params& prm) {
   prm.total_q = p->total_q;
   prm.total_out = p->total_kv_out;
   prm.total_in = p->total_kv_in;
-  prm.tr = pl.tr;
   prm.tiles = pl.tiles;
-  prm.n_groups = pl.n_groups;
   prm.splits = pl.splits;
-  prm.kps = pl.kps;
-  prm.slots = pl.slots;
 }
 
 void fill_workspace(const Plan& pl, void* ws, fb::Params& prm) {
   char* base = static_cast<char*>(ws);
-  prm.group_ctr = reinterpret_cast<int*>(base + pl.off_group_ctr);
   prm.grid_ctr = reinterpret_cast<int*>(base + pl.off_grid_ctr);
   prm.cos = reinterpret_cast<const float*>(base + pl.off_cos);
-  prm.part_a = reinterpret_cast<float*>(base + pl.off_part_a);
-  prm.part_l = reinterpret_cast<float*>(base + pl.off_part_l);
+  prm.ws_in_a = reinterpret_cast<float*>(base + pl.off_in_a);
+  prm.ws_in_l = reinterpret_cast<float*>(base + pl.off_in_l);
 }
 
 }  // namespace
@@ -312,7 +303,7 @@ int32_t fb_version(void) { return 100; }
 fb_status fb_workspace_size(const fb_problem* problem, size_t* bytes) {
   FB_TRY(check_problem(problem));
   if (!bytes) return fail(FB_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = make_plan(problem, device_sms()).bytes;
+  *bytes = make_plan(problem, device_sms(), false).bytes;
   return FB_OK;
 }
 
@@ -335,7 +326,7 @@ fb_status fb_out_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16
   FB_TRY(check_ptr(a_out, "a_out", rows));
   if (rows && !l_out) return fail(FB_ERR_INVALID_ARG, "l_out is NULL");
   if (problem->num_seqs == 0 || !rows) return FB_OK;
-  const Plan pl = make_plan(problem, device_sms());
+  const Plan pl = make_plan(problem, device_sms(), false);
   if (!workspace || workspace_bytes < pl.bytes)
     return fail(FB_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, pl.bytes);
   fb::Params prm;
@@ -349,8 +340,7 @@ fb_status fb_out_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16
   prm.head_mask = head_mask;
   prm.cache_a = a_out;
   prm.cache_l = l_out;
-  prm.n_in_ctas = 0;
-  return launch_attn(pl, prm, pl.n_groups * pl.splits, reinterpret_cast<cudaStream_t>(stream));
+  return launch_attn(pl, prm, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16* k_in, const fb_bf16* v_in,
@@ -363,7 +353,7 @@ fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16*
   FB_TRY(check_ptr(a_in, "a_in", rows));
   if (rows && !l_in) return fail(FB_ERR_INVALID_ARG, "l_in is NULL");
   if (problem->num_seqs == 0 || !rows) return FB_OK;
-  const Plan pl = make_plan(problem, device_sms());
+  const Plan pl = make_plan(problem, device_sms(), true);
   fb::Params prm;
   std::memset(&prm, 0, sizeof(prm));
   fill_problem(problem, pl, prm);
@@ -373,8 +363,7 @@ fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16*
   prm.do_in = 1;
   prm.a_in = a_in;
   prm.l_in = l_in;
-  prm.n_in_ctas = pl.n_groups;
-  return launch_attn(pl, prm, pl.n_groups, reinterpret_cast<cudaStream_t>(stream));
+  return launch_attn(pl, prm, reinterpret_cast<cudaStream_t>(stream));
 }
 
 fb_status fb_merge(int64_t n, int32_t d, const float* a_out, const float* l_out, const float* a_in,
@@ -440,7 +429,7 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   if (problem->num_seqs > 0 && !cache->valid) return fail(FB_ERR_INVALID_ARG, "cache->valid is NULL");
   if (cache->q_ref) FB_TRY(check_ptr(cache->q_ref, "cache->q_ref", true));
   if (problem->num_seqs == 0) return FB_OK;
-  const Plan pl = make_plan(problem, device_sms());
+  const Plan pl = make_plan(problem, device_sms(), false);
   if (!workspace || workspace_bytes < pl.bytes)
     return fail(FB_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, pl.bytes);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -475,8 +464,7 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   prm.a_full = reinterpret_cast<__nv_bfloat16*>(a_full);
   prm.l_full = l_full;
   prm.decision_out = decision_out;
-  prm.n_in_ctas = pl.n_groups;
-  return launch_attn(pl, prm, pl.n_groups * (1 + pl.splits), st);
+  return launch_attn(pl, prm, st);
 }
 
 fb_status fb_cache_invalidate(const fb_problem* problem, const fb_cache* cache, fb_stream_t stream) {

@@ -1,30 +1,35 @@
 // FlashBlock denoise-step attention kernels (sm_100a).
 //
-// One kernel, `attn_kernel`, serves the out-of-block pass, the in-block pass and
-// the fused step.  Its grid holds two kinds of CTAs:
+// `attn_kernel` serves the out-of-block pass (J_out, the cached prefix), the
+// in-block pass (J_in, the block's own tokens, bidirectional) and the fused step.
 //
-//   in-CTAs   one per group (sequence b, kv-head hk, row tile t): softmax
-//             attention of the tile's rows over the block's keys J_in(b);
-//   out-CTAs  `splits` per group: attention over one key range of the prefix
-//             J_out(b), only for groups with a head that recomputes.
+// Work decomposition.  A group is (sequence b, kv-head hk, row tile t); a row is a
+// (query token, q-head of the kv-head's group) pair, so one kv-head's K/V is
+// streamed once for all of its q-heads (grouped-query attention).  Each group is
+// handled by S CTAs that form one thread-block cluster.  The group's prefix key
+// chunks (64 keys each) are dealt out over the S CTAs; the block's chunks, when the
+// block pass runs, go to the last CTA, whose prefix share is shortened to match.
+// Every CTA computes partials (A, L) with A normalised and L = ln Z (FlashBlock,
+// "Mecanismo Central") and keeps them in shared memory: the block partial in a
+// region of its own (the block segment runs first), the prefix partial in the
+// drained stage ring.
 //
-// A "row" of a group is a (query token, q-head of the kv-head's group) pair, so a
-// grouped-query kv-head streams its K/V once for all its q-heads.  Every CTA
-// produces a partial (A, L) for its rows: A normalised, L = ln Z (FlashBlock,
-// "Mecanismo Central").  Partials reach global memory; the last CTA of a group to
-// finish (an atomic counter, no waiting) combines them with the log-space rule
-//   A = sum_s e^{L_s-m} A_s / sum_s e^{L_s-m},  L = m + ln sum_s e^{L_s-m},
-// which is associative, so splitting the prefix and merging the block partial
-// are the same operation.  It stores the recomputed out-of-block partial in the
-// cache, reads the cached one for heads that reuse, and writes A_full / L_full.
-// The last CTA of the whole grid marks recomputed heads valid and writes the
-// decision mask.  No CTA ever waits for another one.
+// Merge.  The log-space composition
+//     A_full = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (e^{L_out-m} + e^{L_in-m})
+// is associative, so combining the S prefix partials and adding the block partial
+// are the same operation.  With S > 1 and a head that recomputes, the cluster
+// synchronises and each CTA merges a slice of the rows, reading the partials of
+// the other CTAs through distributed shared memory; otherwise the CTA that holds
+// all partials merges every row.  The merge writes the cache for heads that
+// recompute, reads it for heads that reuse, and writes A_full / L_full.  No CTA
+// waits on another CTA outside the cluster barriers; the last CTA of the grid (an
+// atomic counter) marks recomputed heads valid and writes the decisions.
 //
-// Inside a CTA: thread 0 streams K/V key tiles with TMA (128-byte swizzle,
-// evict-first L2 policy) through a ring of mbarrier-guarded stages; the WM x WN
-// warps run mma.sync m16n8k16 (bf16 in, fp32 accumulate) with an online softmax
-// in base 2.  Warp (wm, wn) owns 16 rows and
-// a 1/WN share of every key tile; the WN shares are merged through shared memory.
+// Inside a CTA: thread 0 streams K/V chunks with TMA (128-byte swizzle,
+// evict-first L2 policy) through a ring of mbarrier-guarded stages.  Warp
+// (wm, wn) owns 16 rows and a 1/WN share of the keys of every stage and runs
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate) with an online softmax in base 2;
+// the WN shares of a row slab are merged through shared memory.
 #pragma once
 
 #include <limits>
@@ -34,9 +39,9 @@
 namespace fb {
 
 constexpr unsigned kGateTau = 1u, kGateHead = 2u, kForceRecompute = 4u, kForceReuse = 8u;
-constexpr int kBN = 64;      // keys per pipeline stage
-constexpr int kStages = 4;   // pipeline depth
-constexpr int kMaxGroup = 32;
+constexpr int kBN = 64;        // keys per pipeline stage
+constexpr int kMaxGroup = 32;  // q-heads per kv-head
+constexpr int kMaxSplits = 8;  // CTAs per cluster (portable limit)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kNegInf = -std::numeric_limits<float>::infinity();
 
@@ -56,7 +61,7 @@ struct alignas(64) Params {
   const __nv_bfloat16* q;
   int total_q, total_out, total_in;  // host totals: every index is checked against them
   // plan
-  int tr, tiles, n_groups, splits, kps, slots, n_in_ctas;
+  int tiles, splits;
   // mode
   int do_out, do_in, fused, update_state;
   // gates
@@ -78,9 +83,8 @@ struct alignas(64) Params {
   float* a_in;
   float* l_in;
   // workspace
-  float* part_a;
-  float* part_l;
-  int* group_ctr;
+  float* ws_in_a;  // [groups][TR][D] block partial of a group in cluster mode
+  float* ws_in_l;  // [groups][TR]
   int* grid_ctr;
 };
 
@@ -98,22 +102,52 @@ __device__ __forceinline__ bool head_recompute(const Params& p, int b, int h) {
   return !reuse;
 }
 
-template <int D, int WM, int WN>
+// Prefix chunks [a, b) of CTA s of S.  The last CTA also runs `in_chunks` block
+// chunks, so it takes fewer prefix chunks; the rest are spread evenly.
+__device__ __forceinline__ void prefix_range(int s, int S, int out_chunks, int in_chunks, int& a, int& b) {
+  if (S == 1) {
+    a = 0;
+    b = out_chunks;
+    return;
+  }
+  const int per = (out_chunks + in_chunks + S - 1) / S;
+  const int last = min(out_chunks, max(0, per - in_chunks));
+  const int rest = out_chunks - last;
+  if (s == S - 1) {
+    a = rest;
+    b = out_chunks;
+    return;
+  }
+  const int q = rest / (S - 1), r = rest % (S - 1);
+  a = s * q + min(s, r);
+  b = a + q + (s < r ? 1 : 0);
+}
+
+template <int D, int WM, int WN, int STAGES>
 struct Cfg {
   static constexpr int kRows = 16 * WM;
-  static constexpr int kConsumerWarps = WM * WN;
-  static constexpr int kThreads = kConsumerWarps * 32;
-  static constexpr int kKW = kBN / WN;              // keys per warp per stage
-  static constexpr int kTileBytes = kBN * D * 2;    // K (or V) tile of one stage
-  static constexpr int kHalfBytes = kBN * 128;      // one 64-column swizzle span
+  static constexpr int kWarps = WM * WN;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kKW = kBN / WN;            // keys of a stage per warp
+  static constexpr int kTileBytes = kBN * D * 2;  // K (or V) tile of one stage
+  static constexpr int kHalfBytes = kBN * 128;    // one 64-column swizzle span
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStageArea = kStages * kStageBytes;
-  static constexpr int kQStride = D + 8;            // padded Q row, elements
+  static constexpr int kStageArea = STAGES * kStageBytes;
+  static constexpr int kQStride = D + 8;  // padded Q row, elements
   static constexpr int kQBytes = kRows * kQStride * 2;
-  static constexpr int kScratchBytes = WN > 1 ? kConsumerWarps * (D / 2 + 4) * 32 * 4 : 0;
-  static constexpr int kSmem = 1024 + kStageArea + kQBytes + 2 * kStages * 8;
+  static constexpr int kRegs = D / 2 + 4;  // o, m, l of one lane
+  static constexpr int kScratchBytes = (WN - 1) * WM * 32 * kRegs * 4;
+  static constexpr int kPStride = D + 4;  // padded partial row, floats
+  static constexpr int kPartBytes = kRows * kPStride * 4 + kRows * 4;
+  static constexpr int kOffQ = kStageArea;
+  static constexpr int kOffScratch = kOffQ + kQBytes;
+  static constexpr int kOffIn = kOffScratch + kScratchBytes;
+  static constexpr int kOffBar = kOffIn + kPartBytes;
+  static constexpr int kOffPos = kOffBar + 2 * STAGES * 8;
+  static constexpr int kSmem = 1024 + kOffPos + kRows * 4;
   static_assert(kKW % 16 == 0, "keys per warp must be a multiple of 16");
-  static_assert(kScratchBytes <= kStageArea, "combine scratch must fit in the stage ring");
+  static_assert(kPartBytes <= kStageArea, "the prefix partial must fit in the stage ring");
+  static_assert(kPartBytes % 16 == 0 && kOffIn % 16 == 0, "16-byte aligned partials");
   static_assert(D == 64 || D == 128, "head_dim");
 };
 
@@ -123,446 +157,510 @@ __device__ __forceinline__ uint32_t swz(int kr, int dd) {
   return static_cast<uint32_t>((dd >> 6) * (kBN * 128) + kr * 128 + ((((dd & 63) >> 3) ^ (kr & 7)) << 4));
 }
 
-template <int D, int WM, int WN>
-__global__ void __launch_bounds__(Cfg<D, WM, WN>::kThreads, 1) attn_kernel(const __grid_constant__ Params p) {
-  using C = Cfg<D, WM, WN>;
+// Running softmax state of one warp: 16 rows; a thread holds rows lane/4 and lane/4+8.
+template <int D>
+struct Acc {
+  float o[D / 8][4];
+  float m[2];
+  float l[2];  // per-thread partial sums; quad-reduced when finished
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    m[0] = m[1] = kNegInf;
+    l[0] = l[1] = 0.f;
+  }
+};
+
+// KW keys of one stage: S = Q K^T, online softmax, O += P V.  `kr0` is the first
+// key row of the warp inside the stage tile.
+template <int D, int KW>
+__device__ __forceinline__ void consume_keys(Acc<D>& acc, const uint32_t (&qf)[D / 16][4], uint32_t kb, uint32_t vb,
+                                             int kr0, int key0, int k_end, float scale_log2, int lane) {
+  float s[KW / 8][4];
+#pragma unroll
+  for (int n = 0; n < KW / 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+    for (int nb = 0; nb < KW / 16; ++nb) {
+      const int mi = lane >> 3;
+      const int kr = kr0 + nb * 16 + (mi >> 1) * 8 + (lane & 7);
+      const int dd = kk * 16 + (mi & 1) * 8;
+      uint32_t r[4];
+      ldsm_x4(r, kb + swz(kr, dd));
+      mma_bf16_16816(s[2 * nb], qf[kk], r[0], r[1]);
+      mma_bf16_16816(s[2 * nb + 1], qf[kk], r[2], r[3]);
+    }
+  }
+  const bool need_mask = key0 + KW > k_end;
+#pragma unroll
+  for (int n = 0; n < KW / 8; ++n) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float v = s[n][e] * scale_log2;
+      if (need_mask && key0 + n * 8 + 2 * (lane & 3) + (e & 1) >= k_end) v = kNegInf;
+      s[n][e] = v;
+    }
+  }
+  float mx[2] = {acc.m[0], acc.m[1]};
+#pragma unroll
+  for (int n = 0; n < KW / 8; ++n) {
+    mx[0] = fmaxf(mx[0], fmaxf(s[n][0], s[n][1]));
+    mx[1] = fmaxf(mx[1], fmaxf(s[n][2], s[n][3]));
+  }
+  float msafe[2], alpha[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    mx[i] = quad_max(mx[i]);
+    msafe[i] = mx[i] == kNegInf ? 0.f : mx[i];
+    alpha[i] = ex2(acc.m[i] - msafe[i]);
+  }
+  float rs[2] = {0.f, 0.f};
+#pragma unroll
+  for (int n = 0; n < KW / 8; ++n) {
+    s[n][0] = ex2(s[n][0] - msafe[0]);
+    s[n][1] = ex2(s[n][1] - msafe[0]);
+    s[n][2] = ex2(s[n][2] - msafe[1]);
+    s[n][3] = ex2(s[n][3] - msafe[1]);
+    rs[0] += s[n][0] + s[n][1];
+    rs[1] += s[n][2] + s[n][3];
+  }
+  // O only needs rescaling when some row's running max moved (exact either way).
+  if (__any_sync(0xffffffffu, mx[0] != acc.m[0] || mx[1] != acc.m[1])) {
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      acc.o[n][0] *= alpha[0];
+      acc.o[n][1] *= alpha[0];
+      acc.o[n][2] *= alpha[1];
+      acc.o[n][3] *= alpha[1];
+    }
+    acc.l[0] *= alpha[0];
+    acc.l[1] *= alpha[1];
+  }
+  acc.m[0] = mx[0];
+  acc.m[1] = mx[1];
+  acc.l[0] += rs[0];
+  acc.l[1] += rs[1];
+#pragma unroll
+  for (int kb2 = 0; kb2 < KW / 16; ++kb2) {
+    uint32_t a[4];
+    a[0] = pack_bf16x2(s[2 * kb2][0], s[2 * kb2][1]);
+    a[1] = pack_bf16x2(s[2 * kb2][2], s[2 * kb2][3]);
+    a[2] = pack_bf16x2(s[2 * kb2 + 1][0], s[2 * kb2 + 1][1]);
+    a[3] = pack_bf16x2(s[2 * kb2 + 1][2], s[2 * kb2 + 1][3]);
+#pragma unroll
+    for (int np = 0; np < D / 16; ++np) {
+      const int mi = lane >> 3;
+      const int kr = kr0 + kb2 * 16 + (mi & 1) * 8 + (lane & 7);
+      const int dd = np * 16 + (mi >> 1) * 8;
+      uint32_t r[4];
+      ldsm_x4_t(r, vb + swz(kr, dd));
+      mma_bf16_16816(acc.o[2 * np], a, r[0], r[1]);
+      mma_bf16_16816(acc.o[2 * np + 1], a, r[2], r[3]);
+    }
+  }
+}
+
+template <int D, int WM, int WN, int STAGES>
+__global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kernel(const __grid_constant__ Params p) {
+  using C = Cfg<D, WM, WN, STAGES>;
   constexpr int TR = C::kRows;
   constexpr int KW = C::kKW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  __nv_bfloat16* q_s = reinterpret_cast<__nv_bfloat16*>(smem + C::kStageArea);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStageArea + C::kQBytes);
-  uint64_t* empty = full + kStages;
+  __nv_bfloat16* q_s = reinterpret_cast<__nv_bfloat16*>(smem + C::kOffQ);
+  float* scratch = reinterpret_cast<float*>(smem + C::kOffScratch);
+  float* in_part = reinterpret_cast<float*>(smem + C::kOffIn);  // block partial: A [TR][kPStride], L [TR]
+  float* out_part = reinterpret_cast<float*>(stages);            // prefix partial, after the ring drains
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* empty = full + STAGES;
+  int* s_pos = reinterpret_cast<int*>(smem + C::kOffPos);  // block position of each tile row (-1: bad)
   __shared__ uint8_t s_rec[kMaxGroup];
   __shared__ int s_flag;
-  __shared__ int s_abort;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-
-  // ---------------------------------------------------------------- role
-  const int cta = blockIdx.x;
-  const bool is_in = cta < p.n_in_ctas;
-  int gidx, split;
-  if (is_in) {
-    gidx = cta;
-    split = p.splits;  // the block partial uses the last slot of the group
-  } else {
-    const int o = cta - p.n_in_ctas;
-    gidx = o / p.splits;
-    split = o % p.splits;
-  }
+  const int wm = warp % WM;
+  const int wn = warp / WM;
+  const int S = p.splits;
+  const int split = blockIdx.x % S;  // == rank in the cluster
+  const int gidx = blockIdx.x / S;
   const int t = gidx % p.tiles;
   const int bh = gidx / p.tiles;
   const int hk = bh % p.hkv;
   const int b = bh / p.hkv;
   const int g = p.g;
 
+  // ------------------------------------------------------------ group metadata
   const int q0 = p.cu_q[b];
-  const int rows = (p.cu_q[b + 1] - q0) * g;
-  const int row0 = t * TR;
-  const int nrows = min(TR, rows - row0);
+  const int n_q = p.cu_q[b + 1] - q0;
   const int out0 = p.cu_out[b];
   const int n_out = p.cu_out[b + 1] - out0;
   const int in0 = p.cu_in[b];
   const int n_in = p.cu_in[b + 1] - in0;
-  const int n_out_splits = n_out > 0 ? (n_out + p.kps - 1) / p.kps : 1;
-  // Offsets that do not fit the buffers the host described: record and do nothing.
-  const bool ranges_ok = q0 >= 0 && rows >= 0 && q0 + rows / max(g, 1) <= p.total_q && out0 >= 0 && n_out >= 0 &&
-                         out0 + n_out <= p.total_out && in0 >= 0 && n_in >= 0 && in0 + n_in <= p.total_in &&
-                         rows / max(g, 1) <= n_in;
-  if (!ranges_ok && tid == 0 && t == 0 && split == 0) record_status(kDevBadIndex);
-
   if (tid < g) s_rec[tid] = head_recompute(p, b, hk * g + tid) ? 1 : 0;
-  if (tid == 0) s_abort = 0;
+  const bool ranges_ok = q0 >= 0 && n_q >= 0 && q0 + n_q <= p.total_q && out0 >= 0 && n_out >= 0 &&
+                         out0 + n_out <= p.total_out && in0 >= 0 && n_in >= 0 && in0 + n_in <= p.total_in &&
+                         n_q <= n_in;
+  if (!ranges_ok && tid == 0 && t == 0 && split == 0) record_status(kDevBadIndex);
+  const int rows = ranges_ok ? n_q * g : 0;
+  const int row0 = t * TR;
+  const int nrows = max(0, min(TR, rows - row0));
   __syncthreads();
   bool any_rec = false;
   for (int j = 0; j < g; ++j) any_rec |= (s_rec[j] != 0);
 
-  const int expected = (p.do_out && any_rec ? n_out_splits : 0) + (p.fused ? 1 : 0);
-  int k_lo, k_hi;
-  bool work;
-  if (is_in) {
-    k_lo = 0;
-    k_hi = n_in;
-    work = ranges_ok && p.do_in && nrows > 0;
-  } else {
-    k_lo = split * p.kps;
-    k_hi = min(n_out, k_lo + p.kps);
-    work = ranges_ok && p.do_out && nrows > 0 && any_rec && split < n_out_splits;
-  }
-  const bool counted = work && (p.fused || !is_in);  // reaches the group counter
+  // ------------------------------------------------------------ chunk schedule
+  const bool do_out = p.do_out && any_rec;
+  const int out_chunks = do_out ? (n_out + kBN - 1) / kBN : 0;
+  const int in_chunks = p.do_in ? (n_in + kBN - 1) / kBN : 0;
+  int pa, pb;  // my prefix chunks
+  prefix_range(split, S, out_chunks, in_chunks, pa, pb);
+  const bool has_in = p.do_in && split == S - 1;
+  const bool has_out = do_out && (pb > pa || (out_chunks == 0 && split == 0));
+  const bool cluster_mode = S > 1 && do_out;  // uniform over the cluster
+  const bool active = nrows > 0;               // uniform over the cluster
+  // The block segment (if any) runs first; its partial goes to a dedicated
+  // region.  The prefix segment runs last, so its partial can reuse the ring.
+  const int nA = has_in ? in_chunks : 0;
+  const int nB = has_out ? pb - pa : 0;
+  const int n_local = nA + nB;
+  // Which CTA merges which rows: all CTAs of a cluster share the rows; otherwise
+  // the CTA that holds every partial merges them all.
+  const bool merger = cluster_mode || has_in || (S == 1 && has_out);
 
-  if (work) {
-    // ------------------------------------------------------------ Q tile
-    for (int v = tid; v < TR * (D / 8); v += C::kThreads) {
+  if (active && (has_in || has_out || cluster_mode)) {
+    // -------------------------------------------------------- Q rows first
+    // (before the K/V flood, so their loads are not queued behind it)
+    constexpr int kQVec = TR * (D / 8);
+    constexpr int kQPer = (kQVec + C::kThreads - 1) / C::kThreads;
+    uint4 qv[kQPer];
+#pragma unroll
+    for (int k = 0; k < kQPer; ++k) {
+      const int v = tid + k * C::kThreads;
       const int r = v / (D / 8);
       const int c = v % (D / 8);
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (r < nrows) {
+      qv[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (v < kQVec && r < nrows) {
         const int rho = row0 + r;
-        const int it = rho / g;
-        const int h = hk * g + rho % g;
-        val = *reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(q0 + it) * p.hq + h) * D + c * 8);
+        qv[k] = *reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(q0 + rho / g) * p.hq + hk * g + rho % g) * D +
+                                                c * 8);
       }
-      *reinterpret_cast<uint4*>(q_s + r * C::kQStride + c * 8) = val;
     }
+    for (int r = tid; r < TR; r += C::kThreads) {
+      int pos = -1;
+      if (r < nrows) {
+        const int it = (row0 + r) / g;
+        pos = p.q_rows ? p.q_rows[q0 + it] : it;
+        if (pos < 0 || pos >= n_in) {
+          record_status(kDevBadIndex);
+          pos = -1;
+        }
+      }
+      s_pos[r] = pos;
+    }
+    // -------------------------------------------------------- TMA ring
     if (tid == 0) {
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < STAGES; ++s) {
         mbar_init(&full[s], 1);
-        mbar_init(&empty[s], C::kConsumerWarps);
+        mbar_init(&empty[s], C::kWarps);
       }
       fence_barrier_init();
     }
-    __syncthreads();
-
-    const int n_chunks = k_hi > k_lo ? (k_hi - k_lo + kBN - 1) / kBN : 0;
-
-    // Thread 0 issues the TMA copies: the first kStages chunks now, chunk c + kStages
-    // once every warp has released stage c % kStages.
-    const CUtensorMap* tk = is_in ? &p.tm_k_in : &p.tm_k_out;
-    const CUtensorMap* tv = is_in ? &p.tm_v_in : &p.tm_v_out;
-    const int y0 = (is_in ? in0 : out0) + k_lo;
     uint64_t pol = 0;
-    int issued = 0;
     auto issue = [&](int c) {
-      const int st = c % kStages;
+      const bool seg_in = c < nA;
+      const int cc = seg_in ? c : c - nA;
+      const CUtensorMap* tk = seg_in ? &p.tm_k_in : &p.tm_k_out;
+      const CUtensorMap* tv = seg_in ? &p.tm_v_in : &p.tm_v_out;
+      const int y = seg_in ? in0 + cc * kBN : out0 + (pa + cc) * kBN;
+      const int st = c % STAGES;
       mbar_arrive_expect_tx(&full[st], C::kStageBytes);
       uint8_t* kd = stages + st * C::kStageBytes;
       uint8_t* vd = kd + C::kTileBytes;
 #pragma unroll
       for (int hh = 0; hh < D / 64; ++hh) {
-        tma_load_2d(kd + hh * C::kHalfBytes, tk, &full[st], hk * D + hh * 64, y0 + c * kBN, pol);
-        tma_load_2d(vd + hh * C::kHalfBytes, tv, &full[st], hk * D + hh * 64, y0 + c * kBN, pol);
+        tma_load_2d(kd + hh * C::kHalfBytes, tk, &full[st], hk * D + hh * 64, y, pol);
+        tma_load_2d(vd + hh * C::kHalfBytes, tv, &full[st], hk * D + hh * 64, y, pol);
       }
-      ++issued;
     };
-    if (tid == 0 && n_chunks > 0) {
-      prefetch_tensormap(tk);
-      prefetch_tensormap(tv);
+    if (tid == 0 && n_local > 0) {
       pol = l2_policy_evict_first();
-      for (int c = 0; c < min(kStages, n_chunks); ++c) issue(c);
+      for (int c = 0; c < min(STAGES, n_local); ++c) issue(c);
     }
-    {
-      // ---------------------------------------------------------- consumers
-      const int wm = warp % WM;
-      const int wn = warp / WM;
-      const bool rows_active = 16 * wm < nrows;
-      uint32_t qf[D / 16][4];
-      if (rows_active) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          ldsm_x4(qf[kk], smem_u32(q_s + (16 * wm + (lane & 15)) * C::kQStride + kk * 16 + (lane >> 4) * 8));
+    // cached rows this CTA will merge with: bring them into L2 early
+    if (merger && p.fused) {
+      for (int r = tid; r < nrows; r += C::kThreads) {
+        const int rho = row0 + r;
+        if (s_rec[rho % g]) continue;
+        const int it = rho / g;
+        const int pos = p.q_rows ? p.q_rows[q0 + it] : it;
+        if (pos >= 0 && pos < n_in)
+          prefetch_l2(p.cache_a + (static_cast<size_t>(in0 + pos) * p.hq + hk * g + rho % g) * D, D * 4);
       }
-      float o[D / 8][4];
+    }
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-      float m_run[2] = {kNegInf, kNegInf};
-      float l_run[2] = {0.f, 0.f};
-      bool ok = true;
+    for (int k = 0; k < kQPer; ++k) {
+      const int v = tid + k * C::kThreads;
+      if (v < kQVec) *reinterpret_cast<uint4*>(q_s + (v / (D / 8)) * C::kQStride + (v % (D / 8)) * 8) = qv[k];
+    }
+    __syncthreads();
+    // q_ref follows the queries of heads that recompute (fb_step, block owner)
+    if (has_in && p.fused && p.q_ref != nullptr && any_rec) {
+      for (int v = tid; v < nrows * (D / 8); v += C::kThreads) {
+        const int r = v / (D / 8);
+        const int c = v % (D / 8);
+        const int j = (row0 + r) % g;
+        if (!s_rec[j] || s_pos[r] < 0) continue;
+        const size_t e = (static_cast<size_t>(in0 + s_pos[r]) * p.hq + hk * g + j) * D + c * 8;
+        *reinterpret_cast<uint4*>(p.q_ref + e) = *reinterpret_cast<const uint4*>(q_s + r * C::kQStride + c * 8);
+      }
+    }
+    const bool rows_active = 16 * wm < nrows;
+    uint32_t qf[D / 16][4];
+    if (rows_active) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        ldsm_x4(qf[kk], smem_u32(q_s + (16 * wm + (lane & 15)) * C::kQStride + kk * 16 + (lane >> 4) * 8));
+    }
 
-      for (int c = 0; c < n_chunks; ++c) {
-        const int st = c % kStages;
-        if (!mbar_wait(&full[st], (c / kStages) & 1)) {
+    Acc<D> acc;
+    acc.reset();
+    bool ok = true;
+    int issued = min(STAGES, n_local);
+
+    // One segment of chunks [c0, c1) of the local sequence.
+    auto run = [&](int c0, int c1) {
+      for (int c = c0; c < c1 && ok; ++c) {
+        const int st = c % STAGES;
+        // every lane waits; the warp leaves together if the wait ran out
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (c / STAGES) & 1))) {
           record_status(kDevTimeout);
-          s_abort = 1;
           ok = false;
           break;
         }
         if (rows_active) {
+          const bool seg_in = c < nA;
+          const int key0 = (seg_in ? c * kBN : (pa + c - nA) * kBN) + wn * KW;
           const uint32_t kb = smem_u32(stages + st * C::kStageBytes);
-          const uint32_t vb = kb + C::kTileBytes;
-          float s[KW / 8][4];
-#pragma unroll
-          for (int n = 0; n < KW / 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-          // S = Q K^T over this warp's KW keys
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-            for (int nb = 0; nb < KW / 16; ++nb) {
-              const int mi = lane >> 3;
-              const int kr = wn * KW + nb * 16 + (mi >> 1) * 8 + (lane & 7);
-              const int dd = kk * 16 + (mi & 1) * 8;
-              uint32_t r[4];
-              ldsm_x4(r, kb + swz(kr, dd));
-              mma_bf16_16816(s[2 * nb], qf[kk], r[0], r[1]);
-              mma_bf16_16816(s[2 * nb + 1], qf[kk], r[2], r[3]);
-            }
-          }
-          // scale to base 2, mask keys past the range end
-          const int key0 = k_lo + c * kBN + wn * KW;
-          const bool need_mask = key0 + KW > k_hi;
-#pragma unroll
-          for (int n = 0; n < KW / 8; ++n) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float v = s[n][e] * p.scale_log2;
-              if (need_mask && key0 + n * 8 + 2 * (lane & 3) + (e & 1) >= k_hi) v = kNegInf;
-              s[n][e] = v;
-            }
-          }
-          // online softmax
-          float mx[2] = {m_run[0], m_run[1]};
-#pragma unroll
-          for (int n = 0; n < KW / 8; ++n) {
-            mx[0] = fmaxf(mx[0], fmaxf(s[n][0], s[n][1]));
-            mx[1] = fmaxf(mx[1], fmaxf(s[n][2], s[n][3]));
-          }
-          float msafe[2], alpha[2];
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            mx[i] = quad_max(mx[i]);
-            msafe[i] = mx[i] == kNegInf ? 0.f : mx[i];
-            alpha[i] = ex2(m_run[i] - msafe[i]);
-            m_run[i] = mx[i];
-          }
-          float rs[2] = {0.f, 0.f};
-#pragma unroll
-          for (int n = 0; n < KW / 8; ++n) {
-            s[n][0] = ex2(s[n][0] - msafe[0]);
-            s[n][1] = ex2(s[n][1] - msafe[0]);
-            s[n][2] = ex2(s[n][2] - msafe[1]);
-            s[n][3] = ex2(s[n][3] - msafe[1]);
-            rs[0] += s[n][0] + s[n][1];
-            rs[1] += s[n][2] + s[n][3];
-          }
-          l_run[0] = l_run[0] * alpha[0] + rs[0];
-          l_run[1] = l_run[1] * alpha[1] + rs[1];
-#pragma unroll
-          for (int n = 0; n < D / 8; ++n) {
-            o[n][0] *= alpha[0];
-            o[n][1] *= alpha[0];
-            o[n][2] *= alpha[1];
-            o[n][3] *= alpha[1];
-          }
-          // O += P V
-#pragma unroll
-          for (int kb2 = 0; kb2 < KW / 16; ++kb2) {
-            uint32_t a[4];
-            a[0] = pack_bf16x2(s[2 * kb2][0], s[2 * kb2][1]);
-            a[1] = pack_bf16x2(s[2 * kb2][2], s[2 * kb2][3]);
-            a[2] = pack_bf16x2(s[2 * kb2 + 1][0], s[2 * kb2 + 1][1]);
-            a[3] = pack_bf16x2(s[2 * kb2 + 1][2], s[2 * kb2 + 1][3]);
-#pragma unroll
-            for (int np = 0; np < D / 16; ++np) {
-              const int mi = lane >> 3;
-              const int kr = wn * KW + kb2 * 16 + (mi & 1) * 8 + (lane & 7);
-              const int dd = np * 16 + (mi >> 1) * 8;
-              uint32_t r[4];
-              ldsm_x4_t(r, vb + swz(kr, dd));
-              mma_bf16_16816(o[2 * np], a, r[0], r[1]);
-              mma_bf16_16816(o[2 * np + 1], a, r[2], r[3]);
-            }
-          }
+          consume_keys<D, KW>(acc, qf, kb, kb + C::kTileBytes, wn * KW, key0, seg_in ? n_in : n_out, p.scale_log2,
+                              lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);
-        if (tid == 0 && c + kStages < n_chunks) {
-          if (!mbar_wait(&empty[st], (c / kStages) & 1)) {
-            record_status(kDevTimeout);
-            s_abort = 1;
-            ok = false;
-            break;
+        if (warp == 0 && c + STAGES < n_local) {
+          bool refill_ok = true;
+          if (lane == 0) {
+            refill_ok = mbar_wait(&empty[st], (c / STAGES) & 1);
+            if (refill_ok) {
+              issue(c + STAGES);
+              ++issued;
+            }
           }
-          issue(c + kStages);
+          if (!__shfl_sync(0xffffffffu, refill_ok ? 1 : 0, 0)) {
+            record_status(kDevTimeout);
+            ok = false;
+          }
         }
       }
-      // Drain: copies issued but never consumed (only after a timeout) land first.
-      if (tid == 0 && !ok) {
-        for (int c = max(0, issued - kStages); c < issued; ++c)
-          if (!mbar_wait(&full[c % kStages], (c / kStages) & 1)) record_status(kDevTimeout);
-      }
+    };
 
-      l_run[0] = quad_sum(l_run[0]);
-      l_run[1] = quad_sum(l_run[1]);
-
-      // ---------------------------------------------------- merge the WN shares
+    // Close a segment: merge the WN key-shares of every row slab and store the
+    // normalised partial (A, L = ln Z) of the tile in `dst` ([TR][kPStride], then [TR]).
+    auto close = [&](float* dst) {
+      float l_tot[2];
+      l_tot[0] = quad_sum(acc.l[0]);
+      l_tot[1] = quad_sum(acc.l[1]);
       if constexpr (WN > 1) {
         __syncthreads();
-        const bool aborted = s_abort != 0;
-        float* scr = reinterpret_cast<float*>(stages);
-        constexpr int kRegs = D / 2 + 4;
-        float* mine = scr + (wn * WM + wm) * kRegs * 32;
-        if (!aborted && wn > 0) {
+        if (wn > 0) {
+          float* mine = scratch + ((wn - 1) * WM + wm) * C::kRegs * 32;
 #pragma unroll
           for (int n = 0; n < D / 8; ++n)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) mine[(n * 4 + e) * 32 + lane] = o[n][e];
-          mine[(D / 2 + 0) * 32 + lane] = m_run[0];
-          mine[(D / 2 + 1) * 32 + lane] = m_run[1];
-          mine[(D / 2 + 2) * 32 + lane] = l_run[0];
-          mine[(D / 2 + 3) * 32 + lane] = l_run[1];
+            for (int e = 0; e < 4; ++e) mine[(n * 4 + e) * 32 + lane] = acc.o[n][e];
+          mine[(D / 2 + 0) * 32 + lane] = acc.m[0];
+          mine[(D / 2 + 1) * 32 + lane] = acc.m[1];
+          mine[(D / 2 + 2) * 32 + lane] = l_tot[0];
+          mine[(D / 2 + 3) * 32 + lane] = l_tot[1];
         }
         __syncthreads();
-        if (!aborted && wn == 0) {
+        if (wn == 0) {
 #pragma unroll 1
           for (int w2 = 1; w2 < WN; ++w2) {
-            const float* th = scr + (w2 * WM + wm) * kRegs * 32;
+            const float* th = scratch + ((w2 - 1) * WM + wm) * C::kRegs * 32;
             float a1[2], a2[2];
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
               const float m2 = th[(D / 2 + i) * 32 + lane];
               const float l2 = th[(D / 2 + 2 + i) * 32 + lane];
-              const float mn = fmaxf(m_run[i], m2);
+              const float mn = fmaxf(acc.m[i], m2);
               const float ms = mn == kNegInf ? 0.f : mn;
-              a1[i] = ex2(m_run[i] - ms);
+              a1[i] = ex2(acc.m[i] - ms);
               a2[i] = ex2(m2 - ms);
-              l_run[i] = l_run[i] * a1[i] + l2 * a2[i];
-              m_run[i] = mn;
+              l_tot[i] = l_tot[i] * a1[i] + l2 * a2[i];
+              acc.m[i] = mn;
             }
 #pragma unroll
             for (int n = 0; n < D / 8; ++n) {
-              o[n][0] = o[n][0] * a1[0] + th[(n * 4 + 0) * 32 + lane] * a2[0];
-              o[n][1] = o[n][1] * a1[0] + th[(n * 4 + 1) * 32 + lane] * a2[0];
-              o[n][2] = o[n][2] * a1[1] + th[(n * 4 + 2) * 32 + lane] * a2[1];
-              o[n][3] = o[n][3] * a1[1] + th[(n * 4 + 3) * 32 + lane] * a2[1];
+              acc.o[n][0] = acc.o[n][0] * a1[0] + th[(n * 4 + 0) * 32 + lane] * a2[0];
+              acc.o[n][1] = acc.o[n][1] * a1[0] + th[(n * 4 + 1) * 32 + lane] * a2[0];
+              acc.o[n][2] = acc.o[n][2] * a1[1] + th[(n * 4 + 2) * 32 + lane] * a2[1];
+              acc.o[n][3] = acc.o[n][3] * a1[1] + th[(n * 4 + 3) * 32 + lane] * a2[1];
             }
           }
         }
+      } else {
+        __syncthreads();  // the ring may be reused as the destination
       }
-
-      // ---------------------------------------------------- write the partial
-      if (ok && wn == 0 && rows_active) {
+      if (wn == 0) {
+        float* dl = dst + TR * C::kPStride;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int r = 16 * wm + (lane >> 2) + 8 * i;
-          if (r < nrows) {
-            const float l = l_run[i];
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            const float lnat = l > 0.f ? (m_run[i] + log2f(l)) * kLn2 : kNegInf;
-            float* arow;
-            float* lptr;
-            if (is_in && !p.fused) {
-              const int rho = row0 + r;
-              const size_t e = static_cast<size_t>(q0 + rho / g) * p.hq + hk * g + rho % g;
-              arow = p.a_in + e * D;
-              lptr = p.l_in + e;
-            } else {
-              const size_t e = (static_cast<size_t>(gidx) * p.slots + split) * TR + r;
-              arow = p.part_a + e * D;
-              lptr = p.part_l + e;
-            }
+          const float z = l_tot[i];
+          const float inv = z > 0.f ? 1.f / z : 0.f;
 #pragma unroll
-            for (int n = 0; n < D / 8; ++n)
-              *reinterpret_cast<float2*>(arow + n * 8 + 2 * (lane & 3)) =
-                  make_float2(o[n][2 * i] * inv, o[n][2 * i + 1] * inv);
-            if ((lane & 3) == 0) *lptr = lnat;
-          }
+          for (int n = 0; n < D / 8; ++n)
+            *reinterpret_cast<float2*>(dst + r * C::kPStride + n * 8 + 2 * (lane & 3)) =
+                make_float2(acc.o[n][2 * i] * inv, acc.o[n][2 * i + 1] * inv);
+          if ((lane & 3) == 0) dl[r] = z > 0.f ? (acc.m[i] + log2f(z)) * kLn2 : kNegInf;
         }
       }
-    }
+      acc.reset();
+      __syncthreads();  // the partial is complete before any warp reads it
+    };
 
-    // q_ref follows the queries of heads that recompute (in-CTA of fb_step)
-    if (is_in && p.fused && p.q_ref != nullptr) {
-      for (int v = tid; v < nrows * (D / 8); v += C::kThreads) {
-        const int r = v / (D / 8);
-        const int c = v % (D / 8);
-        const int rho = row0 + r;
-        const int j = rho % g;
-        if (!s_rec[j]) continue;
-        const int prow = q0 + rho / g;
-        const int pos = p.q_rows ? p.q_rows[prow] : rho / g;
-        if (pos < 0 || pos >= n_in) {
-          record_status(kDevBadIndex);
-          continue;
-        }
-        const size_t e = (static_cast<size_t>(in0 + pos) * p.hq + hk * g + j) * D + c * 8;
-        *reinterpret_cast<uint4*>(p.q_ref + e) = *reinterpret_cast<const uint4*>(q_s + r * C::kQStride + c * 8);
+    // -------------------------------------------------------- the two segments
+    if (has_in) {
+      run(0, nA);
+      close(in_part);
+    }
+    if (has_out) {
+      run(nA, n_local);
+      // every issued copy has landed before the ring is reused
+      if (tid == 0 && !ok) {
+        for (int c = max(0, issued - STAGES); c < issued; ++c)
+          if (!mbar_wait(&full[c % STAGES], (c / STAGES) & 1)) record_status(kDevTimeout);
       }
+      close(out_part);
+    } else if (tid == 0 && !ok) {
+      for (int c = max(0, issued - STAGES); c < issued; ++c)
+        if (!mbar_wait(&full[c % STAGES], (c / STAGES) & 1)) record_status(kDevTimeout);
     }
-  }
 
-  // ---------------------------------------------------------------- group merge
-  if (counted) {
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_flag = (atomicAdd(&p.group_ctr[gidx], 1) == expected - 1) ? 1 : 0;
-    __syncthreads();
-    if (s_flag) {
-      __threadfence();
-      constexpr int VPT = D / 32;  // floats per lane of one row
-      const int nw = C::kThreads / 32;
-      for (int r = warp; r < nrows; r += nw) {
+    // -------------------------------------------------------- merge
+    if (cluster_mode) cluster_sync();
+    if (merger) {
+      const int rp = cluster_mode ? (nrows + S - 1) / S : nrows;
+      const int r_lo = cluster_mode ? split * rp : 0;
+      const int r_hi = min(nrows, r_lo + rp);
+      const uint32_t out_l = smem_u32(out_part);
+      const uint32_t in_l = smem_u32(in_part);
+      constexpr int kC4 = D / 4;  // float4 columns of a row
+      // owners of prefix partials (same schedule on every CTA of the cluster)
+      uint32_t owners = 0;
+      for (int s2 = 0; s2 < S; ++s2) {
+        int a0, a1;
+        prefix_range(s2, S, out_chunks, in_chunks, a0, a1);
+        if (a1 > a0) owners |= 1u << s2;
+      }
+      for (int item = tid; item < (r_hi - r_lo) * kC4; item += C::kThreads) {
+        const int r = r_lo + item / kC4;
+        const int c4 = (item % kC4) * 4;
+        const int pos = s_pos[r];
+        if (pos < 0) continue;
         const int rho = row0 + r;
-        const int it = rho / g;
         const int j = rho % g;
         const int h = hk * g + j;
-        const int prow = q0 + it;
-        const int pos = p.q_rows ? p.q_rows[prow] : it;
-        if (pos < 0 || pos >= n_in) {
-          record_status(kDevBadIndex);
-          continue;
-        }
         const size_t ce = static_cast<size_t>(in0 + pos) * p.hq + h;
-        float ao[VPT];
-        float lo = kNegInf;
-#pragma unroll
-        for (int v = 0; v < VPT; ++v) ao[v] = 0.f;
         const bool rec = s_rec[j] != 0;
-        if (p.do_out && rec) {
-          const size_t base = static_cast<size_t>(gidx) * p.slots * TR + r;
+        float4 ao = make_float4(0.f, 0.f, 0.f, 0.f);
+        float lo = kNegInf;
+        if (do_out && rec) {
+          // prefix partials of the owners: all loads first, then the log-space sum
+          float ls[kMaxSplits];
+          float4 as[kMaxSplits];
+#pragma unroll
+          for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+            ls[s2] = kNegInf;
+            if (s2 < S && (owners >> s2 & 1u)) {
+              const uint32_t rank = cluster_mode ? s2 : split;
+              const uint32_t lb = out_l + (TR * C::kPStride + r) * 4;
+              const uint32_t ab = out_l + (r * C::kPStride + c4) * 4;
+              ls[s2] = cluster_mode ? ld_dsmem_f32(dsmem_addr(lb, rank)) : out_part[TR * C::kPStride + r];
+              as[s2] = cluster_mode ? ld_dsmem_f4(dsmem_addr(ab, rank))
+                                    : *reinterpret_cast<const float4*>(out_part + r * C::kPStride + c4);
+            }
+          }
           float mx = kNegInf;
-          for (int s2 = 0; s2 < n_out_splits; ++s2) mx = fmaxf(mx, __ldcg(p.part_l + base + s2 * TR));
+#pragma unroll
+          for (int s2 = 0; s2 < kMaxSplits; ++s2) mx = fmaxf(mx, ls[s2]);
           if (mx != kNegInf) {
             float den = 0.f;
-            for (int s2 = 0; s2 < n_out_splits; ++s2) {
-              const float ls = __ldcg(p.part_l + base + s2 * TR);
-              const float w = ls == kNegInf ? 0.f : expf(ls - mx);
-              den += w;
-              const float* src = p.part_a + (base + s2 * TR) * D + lane * VPT;
 #pragma unroll
-              for (int v = 0; v < VPT; ++v) ao[v] += w * __ldcg(src + v);
+            for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+              if (ls[s2] == kNegInf) continue;
+              const float w = expf(ls[s2] - mx);
+              den += w;
+              ao.x += w * as[s2].x;
+              ao.y += w * as[s2].y;
+              ao.z += w * as[s2].z;
+              ao.w += w * as[s2].w;
             }
             const float inv = 1.f / den;
-#pragma unroll
-            for (int v = 0; v < VPT; ++v) ao[v] *= inv;
+            ao.x *= inv;
+            ao.y *= inv;
+            ao.z *= inv;
+            ao.w *= inv;
             lo = mx + logf(den);
           }
-#pragma unroll
-          for (int v = 0; v < VPT; ++v) p.cache_a[ce * D + lane * VPT + v] = ao[v];
-          if (lane == 0) p.cache_l[ce] = lo;
+          *reinterpret_cast<float4*>(p.cache_a + ce * D + c4) = ao;
+          if (c4 == 0) p.cache_l[ce] = lo;
         } else if (p.fused) {
-#pragma unroll
-          for (int v = 0; v < VPT; ++v) ao[v] = p.cache_a[ce * D + lane * VPT + v];
+          ao = *reinterpret_cast<const float4*>(p.cache_a + ce * D + c4);
           lo = p.cache_l[ce];
         }
-        if (p.fused) {
-          const size_t ie = (static_cast<size_t>(gidx) * p.slots + p.splits) * TR + r;
-          const float li = __ldcg(p.part_l + ie);
-          const float* ai = p.part_a + ie * D + lane * VPT;
-          const float mx = fmaxf(lo, li);
-          float af[VPT];
-          float lf = kNegInf;
-          if (mx == kNegInf) {
-#pragma unroll
-            for (int v = 0; v < VPT; ++v) af[v] = 0.f;
+        if (p.do_in) {
+          // the block partial lives in the last CTA of the cluster
+          const uint32_t rank = S - 1;
+          const float li = cluster_mode ? ld_dsmem_f32(dsmem_addr(in_l + (TR * C::kPStride + r) * 4, rank))
+                                        : in_part[TR * C::kPStride + r];
+          const float4 ai = cluster_mode ? ld_dsmem_f4(dsmem_addr(in_l + (r * C::kPStride + c4) * 4, rank))
+                                         : *reinterpret_cast<const float4*>(in_part + r * C::kPStride + c4);
+          const size_t fe = static_cast<size_t>(q0 + rho / g) * p.hq + h;
+          if (!p.fused) {
+            *reinterpret_cast<float4*>(p.a_in + fe * D + c4) = ai;
+            if (c4 == 0) p.l_in[fe] = li;
           } else {
-            const float wo = lo == kNegInf ? 0.f : expf(lo - mx);
-            const float wi = li == kNegInf ? 0.f : expf(li - mx);
-            const float den = wo + wi;
-            const float inv = 1.f / den;
-#pragma unroll
-            for (int v = 0; v < VPT; ++v) af[v] = (wo * ao[v] + wi * __ldcg(ai + v)) * inv;
-            lf = mx + logf(den);
+            const float mx = fmaxf(lo, li);
+            float wo = 0.f, wi = 0.f, lf = kNegInf;
+            if (mx != kNegInf) {
+              wo = lo == kNegInf ? 0.f : expf(lo - mx);
+              wi = li == kNegInf ? 0.f : expf(li - mx);
+              const float den = wo + wi;
+              lf = mx + logf(den);
+              wo /= den;
+              wi /= den;
+            }
+            __nv_bfloat16* dst = p.a_full + fe * D + c4;
+            *reinterpret_cast<__nv_bfloat162*>(dst) =
+                __floats2bfloat162_rn(wo * ao.x + wi * ai.x, wo * ao.y + wi * ai.y);
+            *reinterpret_cast<__nv_bfloat162*>(dst + 2) =
+                __floats2bfloat162_rn(wo * ao.z + wi * ai.z, wo * ao.w + wi * ai.w);
+            if (c4 == 0 && p.l_full) p.l_full[fe] = lf;
           }
-          const size_t fe = static_cast<size_t>(prow) * p.hq + h;
-          __nv_bfloat16* dst = p.a_full + fe * D + lane * VPT;
-#pragma unroll
-          for (int v = 0; v < VPT; v += 2)
-            *reinterpret_cast<__nv_bfloat162*>(dst + v) = __floats2bfloat162_rn(af[v], af[v + 1]);
-          if (lane == 0 && p.l_full) p.l_full[fe] = lf;
         }
       }
-      if (tid == 0) p.group_ctr[gidx] = 0;
     }
+    if (cluster_mode) cluster_sync();  // no CTA leaves while its partials may still be read
   }
 
-  // ---------------------------------------------------------------- grid epilogue
+  // ------------------------------------------------------------ grid epilogue
   if (p.update_state) {
     __syncthreads();
-    __threadfence();
     if (tid == 0) s_flag = (atomicAdd(p.grid_ctr, 1) == static_cast<int>(gridDim.x) - 1) ? 1 : 0;
     __syncthreads();
     if (s_flag) {
