@@ -2,25 +2,32 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
                     [--workload dllm_layer|long_context_gqa|varlen_branches|video|tiny]
+                    [--layers L]
 
-One bench step is one denoise episode of the workload's block (32 denoise steps
-for the 8B-dLLM layer: the cache is invalidated, step 0 recomputes, later steps
-follow the tau gate).  Every denoise step is one fb_step call (gates, out-of-block
-pass when recomputing, in-block pass, log-space merge) on resident inputs, timed
-with CUDA events on the launching stream; L2 is flushed (a 256 MiB read) before
-every denoise step and the flush is not timed.  `value` is the mean denoise-step
-latency in microseconds over the K timed episodes (max over ranks).
+The workload is run the way a block-diffusion model runs it: every denoise step
+calls the attention of each of L layers (32 for the 8B dLLM), and every layer has
+its own prefix K/V, FlashBlock cache and block inputs (distinct device buffers;
+the prefixes alone are L x 64 MiB = 2 GiB for the 8B-dLLM layer, far above L2).
+L2 is flushed (a 256 MiB read, untimed) before every denoise step, so each call
+starts with its data cold.  The L calls of a denoise step are replayed as one CUDA
+graph and timed with CUDA events on the launching stream.
+
+One bench step is one denoise episode of the block: the caches are invalidated
+(untimed set-up of a new block), step 0 recomputes, later steps follow the workload's reuse gates (32 denoise
+steps x L layers = 1024 fb_step calls for the 8B-dLLM layer).  `value` is the
+mean latency of one attention call (one layer, one denoise step) in microseconds
+over the K timed episodes (max over ranks).
 
 `e2e` is the same metric through the public API with host buffers: each denoise
-step copies its block Q/K/V and update count from pinned host memory, calls
-fb_step and copies A_full and L_full back, all inside the timed region.
+step's graph also copies every layer's block Q/K/V and update count from pinned
+host memory and copies A_full and L_full back.
 
-`roofline` is the fused attention kernel on its recompute launches (the prefix
-pass: HBM-bound), with achieved = algorithmic bytes / launch time;
-`roofline_all_launches` aggregates every launch of the episode.
+`roofline` is the fused attention kernel on its recompute launches (prefix pass +
+block pass + merge; HBM-bound), achieved = algorithmic bytes per launch / launch
+time on recompute steps; `roofline_all_launches` aggregates every launch.
 
 `--impl reference` times the fp64 oracle (the plain CPU statement of the method)
-on the host cores on the same workload, one episode per step, rank 0 only.
+on the host cores on one layer of the same workload, rank 0 only.
 
 With torchrun (N > 1) every rank runs its own request (seed + rank) on its own
 GPU with no collective on the data path (weak scaling); ranks meet only at the
@@ -179,100 +186,130 @@ def make_workload(name: str, seed: int):
 
 # ---------------------------------------------------------------- native arm
 
-class Episode:
-    """Device-resident inputs and buffers for one workload, run through fb_step."""
+DEFAULT_LAYERS = {"dllm_layer": 32, "long_context_gqa": 2, "varlen_branches": 32, "video": 8, "tiny": 32}
 
-    def __init__(self, w, device):
+
+class Model:
+    """L layers of one workload shape on the device, run through fb_step.
+
+    Layer l holds its own copies of the prefix K/V, the block inputs of every
+    step, the FlashBlock cache, the workspace and the outputs."""
+
+    def __init__(self, w, layers, device):
         import torch
         from cached_split_attention_b200 import binding as B
-        self.torch, self.B = torch, B
-        self.w = w
-        self.device = device
+        self.torch, self.B, self.w, self.L = torch, B, w, layers
+        S = len(w.steps)
+        self.S = S
         p = w.problem
         self.dp = [B.DeviceProblem(st.problem, device) for st in w.steps]
-        self.cache = B.Cache(p, device, with_q_ref=bool(w.flags & W.GATE_HEAD))
-        self.k_out = B.bf16_tensor(w.k_out, device)
-        self.v_out = B.bf16_tensor(w.v_out, device)
-        self.q = [B.bf16_tensor(st.q, device) for st in w.steps]
-        self.k_in = [B.bf16_tensor(st.k_in, device) for st in w.steps]
-        self.v_in = [B.bf16_tensor(st.v_in, device) for st in w.steps]
-        self.n_upd = [torch.as_tensor(st.n_updated, dtype=torch.int32).to(device) for st in w.steps]
         wsz = max(B.workspace_size(d) for d in self.dp)
-        self.ws = torch.empty(wsz, dtype=torch.uint8, device=device)
-        B.workspace_init(self.ws)
+        k_out0, v_out0 = B.bf16_tensor(w.k_out, device), B.bf16_tensor(w.v_out, device)
+        q0 = [B.bf16_tensor(st.q, device) for st in w.steps]
+        ki0 = [B.bf16_tensor(st.k_in, device) for st in w.steps]
+        vi0 = [B.bf16_tensor(st.v_in, device) for st in w.steps]
+        n0 = [torch.as_tensor(st.n_updated, dtype=torch.int32).to(device) for st in w.steps]
         H, d = p.num_heads_q, p.head_dim
         tq = max(st.problem.total_q for st in w.steps)
-        self.a_full = torch.empty((tq, H, d), dtype=torch.bfloat16, device=device)
-        self.l_full = torch.empty((tq, H), dtype=torch.float32, device=device)
-        self.dec = torch.empty((p.num_seqs, H), dtype=torch.uint8, device=device)
-        self.prm = B.params(w.tau, w.gamma, w.flags)
-        # pinned host copies for the end-to-end leg
+        self.layers = []
+        for _ in range(layers):
+            lay = dict(
+                k_out=k_out0.clone(), v_out=v_out0.clone(),
+                q=[x.clone() for x in q0], k_in=[x.clone() for x in ki0], v_in=[x.clone() for x in vi0],
+                n=[x.clone() for x in n0],
+                cache=B.Cache(p, device, with_q_ref=bool(w.flags & W.GATE_HEAD)),
+                ws=torch.empty(wsz, dtype=torch.uint8, device=device),
+                a_full=torch.empty((tq, H, d), dtype=torch.bfloat16, device=device),
+                l_full=torch.empty((tq, H), dtype=torch.float32, device=device),
+                dec=torch.empty((p.num_seqs, H), dtype=torch.uint8, device=device))
+            B.workspace_init(lay["ws"])
+            self.layers.append(lay)
+        del k_out0, v_out0, q0, ki0, vi0, n0
+        # pinned host copies for the end-to-end leg (shared by the layers)
         self.h_q = [torch.from_numpy(st.q.view(np.int16)).pin_memory() for st in w.steps]
         self.h_k = [torch.from_numpy(st.k_in.view(np.int16)).pin_memory() for st in w.steps]
         self.h_v = [torch.from_numpy(st.v_in.view(np.int16)).pin_memory() for st in w.steps]
         self.h_n = [torch.from_numpy(st.n_updated.astype(np.int32)).pin_memory() for st in w.steps]
-        self.d_q = torch.empty_like(self.q[0]).view(torch.int16)
-        self.d_k = torch.empty_like(self.k_in[0]).view(torch.int16)
-        self.d_v = torch.empty_like(self.v_in[0]).view(torch.int16)
-        self.d_n = torch.empty_like(self.n_upd[0])
-        self.h_a = torch.empty(self.a_full.shape, dtype=torch.bfloat16).pin_memory()
-        self.h_l = torch.empty(self.l_full.shape, dtype=torch.float32).pin_memory()
-        # L2 flush: read 256 MiB (about twice the L2) so that the next step starts
-        # with none of its data in L2 and no dirty lines to write back
+        self.h_a = [torch.empty((tq, H, d), dtype=torch.bfloat16).pin_memory() for _ in range(layers)]
+        self.h_l = [torch.empty((tq, H), dtype=torch.float32).pin_memory() for _ in range(layers)]
+        # L2 flush: read 256 MiB (about twice the L2)
         self.flush_buf = torch.ones(64 << 20, dtype=torch.int32, device=device)
         self.flush_out = torch.empty((), dtype=torch.int32, device=device)
+        self.graphs = {}
 
-    def step(self, s, stream):
-        B = self.B
-        B.step(self.dp[s], self.prm, self.cache, self.q[s], self.k_in[s], self.v_in[s], self.k_out, self.v_out,
-               self.n_upd[s], self.a_full, self.ws, l_full=self.l_full, decision_out=self.dec, stream=stream)
-
-    def step_e2e(self, s, stream):
+    def call(self, li, s, prm, stream, e2e=False):
         torch, B = self.torch, self.B
-        with torch.cuda.stream(stream):
-            self.d_q.copy_(self.h_q[s], non_blocking=True)
-            self.d_k.copy_(self.h_k[s], non_blocking=True)
-            self.d_v.copy_(self.h_v[s], non_blocking=True)
-            self.d_n.copy_(self.h_n[s], non_blocking=True)
-            B.step(self.dp[s], self.prm, self.cache, self.d_q.view(torch.bfloat16), self.d_k.view(torch.bfloat16),
-                   self.d_v.view(torch.bfloat16), self.k_out, self.v_out, self.d_n, self.a_full, self.ws,
-                   l_full=self.l_full, decision_out=self.dec, stream=stream)
+        lay = self.layers[li]
+        if e2e:
+            lay["q"][s].view(torch.int16).copy_(self.h_q[s], non_blocking=True)
+            lay["k_in"][s].view(torch.int16).copy_(self.h_k[s], non_blocking=True)
+            lay["v_in"][s].view(torch.int16).copy_(self.h_v[s], non_blocking=True)
+            lay["n"][s].copy_(self.h_n[s], non_blocking=True)
+        B.step(self.dp[s], prm, lay["cache"], lay["q"][s], lay["k_in"][s], lay["v_in"][s], lay["k_out"],
+               lay["v_out"], lay["n"][s], lay["a_full"], lay["ws"], l_full=lay["l_full"], decision_out=lay["dec"],
+               stream=stream)
+        if e2e:
             tq = self.dp[s].host.total_q
-            self.h_a[:tq].copy_(self.a_full[:tq], non_blocking=True)
-            self.h_l[:tq].copy_(self.l_full[:tq], non_blocking=True)
+            self.h_a[li][:tq].copy_(lay["a_full"][:tq], non_blocking=True)
+            self.h_l[li][:tq].copy_(lay["l_full"][:tq], non_blocking=True)
+
+    def denoise_step(self, s, prm, stream, e2e=False):
+        """Attention of every layer for denoise step s."""
+        for li in range(self.L):
+            self.call(li, s, prm, stream, e2e)
+
+    def new_block(self, stream):
+        """A new block starts: every layer's cache is empty (episode set-up, untimed)."""
+        for lay in self.layers:
+            self.B.cache_invalidate(self.dp[0], lay["cache"], stream=stream)
+
+    def graph(self, s, flags, e2e):
+        key = (s, flags, e2e)
+        if key not in self.graphs:
+            torch = self.torch
+            prm = self.B.params(self.w.tau, self.w.gamma, flags)
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                self.denoise_step(s, prm, side, e2e)  # warm-up outside capture
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.denoise_step(s, prm, torch.cuda.current_stream(), e2e)
+            torch.cuda.synchronize()
+            self.graphs[key] = (g, prm)
+        return self.graphs[key][0]
+
+    def episode(self, flags, events=None, e2e=False):
+        torch = self.torch
+        stream = torch.cuda.current_stream()
+        for s in range(self.S):
+            g = self.graph(s, flags, e2e)
+            if s == 0:
+                self.new_block(stream)
+            torch.amax(self.flush_buf, dim=0, out=self.flush_out)
+            if events is not None:
+                events[s][0].record(stream)
+            g.replay()
+            if events is not None:
+                events[s][1].record(stream)
 
     def e2e_bytes(self, s):
         st = self.w.steps[s]
         tq = st.problem.total_q
         H, d = self.w.problem.num_heads_q, self.w.problem.head_dim
-        return st.q.nbytes + st.k_in.nbytes + st.v_in.nbytes + st.n_updated.astype(np.int32).nbytes, \
-            tq * H * d * 2 + tq * H * 4
+        return (st.q.nbytes + st.k_in.nbytes + st.v_in.nbytes + st.n_updated.astype(np.int32).nbytes,
+                tq * H * d * 2 + tq * H * 4)
 
-    def flush(self, stream):
-        with self.torch.cuda.stream(stream):
-            self.torch.amax(self.flush_buf, dim=0, out=self.flush_out)
 
-    def run_episode(self, stream, events=None, e2e=False, flags=None):
-        """All denoise steps of the episode; events[s] = (start, end) per step."""
-        B = self.B
-        if flags is not None:
-            self.prm = B.params(self.w.tau, self.w.gamma, flags)
-        B.cache_invalidate(self.dp[0], self.cache, stream=stream)
-        decisions = []
-        for s in range(len(self.w.steps)):
-            self.flush(stream)
-            if events is not None:
-                events[s][0].record(stream)
-            if e2e:
-                self.step_e2e(s, stream)
-            else:
-                self.step(s, stream)
-            if events is not None:
-                events[s][1].record(stream)
-            decisions.append(None)
-        if flags is not None:
-            self.prm = B.params(self.w.tau, self.w.gamma, self.w.flags)
-        return decisions
+def _events(torch, K, S):
+    return [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
+            for _ in range(K)]
+
+
+def _elapsed_us(ev):
+    return np.array([[e0.elapsed_time(e1) * 1e3 for e0, e1 in row] for row in ev])
 
 
 def native(args, world, rank, local):
@@ -286,73 +323,71 @@ def native(args, world, rank, local):
     base = {"tiny": 1000, "dllm_layer": 1001, "long_context_gqa": 1002, "varlen_branches": 1003,
             "video": 1004}[args.workload]
     w = make_workload(args.workload, shard_seed(base, rank))
-    ep = Episode(w, device)
-    stream = torch.cuda.current_stream(device)
-    S = len(w.steps)
+    L = args.layers or DEFAULT_LAYERS[args.workload]
+    model = Model(w, L, device)
+    S = model.S
     p = w.problem
 
-    # The decisions of the episode (deterministic): run once to read them.
-    decisions = []
-    ep.B.cache_invalidate(ep.dp[0], ep.cache, stream=stream)
+    # decisions of the episode (identical for every layer): one eager pass
+    stream = torch.cuda.current_stream()
+    prm = model.B.params(w.tau, w.gamma, w.flags)
+    lay0 = model.layers[0]
+    model.B.cache_invalidate(model.dp[0], lay0["cache"], stream=stream)
+    rec_frac = []
     for s in range(S):
-        ep.step(s, stream)
-        decisions.append(ep.dec.cpu().numpy().astype(bool).copy())
-    rec_frac = [float(d.mean()) for d in decisions]
+        model.call(0, s, prm, stream)
+        rec_frac.append(float(lay0["dec"].float().mean().item()))
 
-    # warm-up episodes
     for _ in range(args.warmup):
-        ep.run_episode(stream)
+        model.episode(w.flags)
     torch.cuda.synchronize()
 
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
-          for _ in range(args.steps)]
+    ev = _events(torch, args.steps, S)
     sampler = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
     with sampler:
         for k in range(args.steps):
-            ep.run_episode(stream, events=ev[k])
+            model.episode(w.flags, events=ev[k])
         torch.cuda.synchronize()
     barrier(world)
-    step_ms = np.array([[ev[k][s][0].elapsed_time(ev[k][s][1]) for s in range(S)] for k in range(args.steps)])
-    episode_ms = float(step_ms.sum(axis=1).mean())
-    mean_step_us = float(step_ms.mean() * 1e3)
+    step_us = _elapsed_us(ev)                       # [K, S]: L calls each
+    call_us = float(step_us.mean() / L)
+    episode_ms = float(step_us.sum(axis=1).mean() * 1e-3)
 
-    # end-to-end leg (host buffers, copies inside the timed region)
-    ev2 = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
-           for _ in range(args.steps)]
-    ep.run_episode(stream, e2e=True)
+    # end-to-end leg: host buffers, copies inside every step's graph
+    ev2 = _events(torch, args.steps, S)
+    model.episode(w.flags, e2e=True)
     torch.cuda.synchronize()
     barrier(world)
     for k in range(args.steps):
-        ep.run_episode(stream, events=ev2[k], e2e=True)
+        model.episode(w.flags, events=ev2[k], e2e=True)
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = np.array([[ev2[k][s][0].elapsed_time(ev2[k][s][1]) for s in range(S)] for k in range(args.steps)])
-    e2e_us = float(e2e_ms.mean() * 1e3)
-    h2d = sum(ep.e2e_bytes(s)[0] for s in range(S)) / S
-    d2h = sum(ep.e2e_bytes(s)[1] for s in range(S)) / S
+    e2e_call_us = float(_elapsed_us(ev2).mean() / L)
+    h2d = sum(model.e2e_bytes(s)[0] for s in range(S)) / S
+    d2h = sum(model.e2e_bytes(s)[1] for s in range(S)) / S
 
-    # dense (forced recompute) and reuse (forced reuse) step latencies, L2 flushed
-    reps = max(3, min(args.steps, 20))
-    evd = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
-           for _ in range(reps)]
-    evr = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(S)]
-           for _ in range(reps)]
+    # dense (forced recompute) and reuse (forced reuse) calls
+    reps = max(3, min(args.steps, 10))
+    evd, evr = _events(torch, reps, S), _events(torch, reps, S)
+    model.episode(W.FORCE_RECOMPUTE)
+    model.episode(W.FORCE_REUSE)
     for k in range(reps):
-        ep.run_episode(stream, events=evd[k], flags=W.FORCE_RECOMPUTE)
+        model.episode(W.FORCE_RECOMPUTE, events=evd[k])
     for k in range(reps):
-        ep.run_episode(stream, events=evr[k], flags=W.FORCE_REUSE)
+        model.episode(W.FORCE_REUSE, events=evr[k])
     torch.cuda.synchronize()
-    dense_us = np.array([[evd[k][s][0].elapsed_time(evd[k][s][1]) * 1e3 for s in range(S)] for k in range(reps)])
-    reuse_us = np.array([[evr[k][s][0].elapsed_time(evr[k][s][1]) * 1e3 for s in range(1, S)] for k in range(reps)])
+    dense_us = _elapsed_us(evd) / L
+    reuse_us = _elapsed_us(evr)[:, 1:] / L
 
-    # roofline of the fused kernel: recompute launches of the timed episodes
+    # roofline of the fused kernel on the recompute steps of the timed episodes
     rec_steps = [s for s in range(S) if rec_frac[s] > 0]
-    bytes_rec = sum(step_bytes(w.steps[s].problem, rec_frac[s])["total"] for s in rec_steps)
-    t_rec = step_ms[:, rec_steps].sum(axis=1).mean() * 1e-3 if rec_steps else float("nan")
+    bytes_rec = [step_bytes(w.steps[s].problem, rec_frac[s])["total"] for s in rec_steps]
+    t_rec = step_us[:, rec_steps].mean(axis=0) / L * 1e-6 if rec_steps else np.array([np.nan])
+    ach_rec = float(np.sum(bytes_rec) / np.sum(t_rec) / 1e9) if rec_steps else float("nan")
     bytes_all = sum(step_bytes(w.steps[s].problem, rec_frac[s])["total"] for s in range(S))
-    t_all = episode_ms * 1e-3
+    ach_all = bytes_all / (episode_ms * 1e-3 / L) / 1e9
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -360,8 +395,6 @@ def native(args, world, rank, local):
         pass
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
-    ach_rec = bytes_rec / t_rec / 1e9 if rec_steps else float("nan")
-    ach_all = bytes_all / t_all / 1e9
     traffic = None
     try:
         prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
@@ -370,8 +403,8 @@ def native(args, world, rank, local):
     except Exception:
         pass
 
-    value = max_over_ranks(mean_step_us, world, device)
-    e2e_v = max_over_ranks(e2e_us, world, device)
+    value = max_over_ranks(call_us, world, device)
+    e2e_v = max_over_ranks(e2e_call_us, world, device)
     ms_step = max_over_ranks(episode_ms, world, device)
     clocks = sampler.summary()
     if rank != 0:
@@ -382,10 +415,11 @@ def native(args, world, rank, local):
     reuse_b = step_bytes(p, 0.0)["total"]
     dense_med = float(np.median(dense_us))
     reuse_med = float(np.median(reuse_us))
+    n_launch = args.steps * S * L * (2 if w.flags & W.GATE_HEAD else 1)
     out = {
         "metric": METRIC,
         "value": round(value, 3),
-        "unit": "us/denoise-step",
+        "unit": "us/attention-call (one layer, one denoise step)",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -397,33 +431,36 @@ def native(args, world, rank, local):
         "data": "synthetic",
         "config": {
             "workload": WORKLOAD_DESC[args.workload],
-            "bench_step": f"one denoise episode ({S} fb_step calls, cache invalidated at its start)",
-            "denoise_steps_per_episode": S,
+            "layers": L,
+            "bench_step": f"one denoise episode: {S} denoise steps x {L} layers = {S * L} fb_step calls",
             "recompute_steps_per_episode": len(rec_steps),
-            "l2": "flushed before every denoise step (256 MiB read, untimed)",
+            "l2": "flushed before every denoise step (256 MiB read, untimed); each layer's data is distinct",
+            "launch": "each denoise step's L calls replayed as one CUDA graph",
             "parallelism": f"replicas x{world} (one request per GPU, no collective)",
             "seed": shard_seed(base, rank),
         },
-        "throughput": {"denoise_steps_per_s_all_gpus": round(world * 1e6 / value, 1)},
-        "dense_step_us": {"median": round(dense_med, 3), "p10": round(float(np.percentile(dense_us, 10)), 3),
+        "throughput": {"attention_calls_per_s_all_gpus": round(world * 1e6 / value, 1)},
+        "dense_call_us": {"median": round(dense_med, 3), "p10": round(float(np.percentile(dense_us, 10)), 3),
                           "p90": round(float(np.percentile(dense_us, 90)), 3),
                           "effective_tbps": round(dense_b / dense_med / 1e6, 3),
                           "frac_of_hbm": round(dense_b / dense_med / 1e3 / hbm_peak, 4)},
-        "reuse_step_us": {"median": round(reuse_med, 3), "p10": round(float(np.percentile(reuse_us, 10)), 3),
+        "reuse_call_us": {"median": round(reuse_med, 3), "p10": round(float(np.percentile(reuse_us, 10)), 3),
                           "p90": round(float(np.percentile(reuse_us, 90)), 3),
                           "effective_tbps": round(reuse_b / reuse_med / 1e6, 3)},
         "reuse_gain": {"predicted_bytes_ratio": round(dense_b / reuse_b, 2),
                        "achieved_time_ratio": round(dense_med / reuse_med, 2)},
-        "roofline": {"bound": "hbm", "kernel": "attn_kernel (recompute launches: prefix pass + block pass + merge)",
+        "roofline": {"bound": "hbm", "kernel": "attn_kernel, recompute launches (prefix + block pass + merge)",
                      "achieved": round(ach_rec, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(ach_rec / hbm_peak, 4), "peak_source": peak_src, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": round(bytes_rec / max(1, len(rec_steps))),
-                     "launches": len(rec_steps) * args.steps},
-        "roofline_all_launches": {"achieved": round(ach_all, 1), "unit": "GB/s", "frac": round(ach_all / hbm_peak, 4),
-                                  "algorithmic_bytes_per_episode": round(bytes_all)},
-        "e2e": {"value": round(e2e_v, 3), "unit": "us/denoise-step", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": int(args.steps * S * (2 if w.flags & W.GATE_HEAD else 1)),
+                     "algorithmic_bytes_per_launch": round(float(np.mean(bytes_rec))) if rec_steps else None,
+                     "launches": len(rec_steps) * L * args.steps},
+        "roofline_all_launches": {"achieved": round(ach_all, 1), "unit": "GB/s",
+                                  "frac": round(ach_all / hbm_peak, 4),
+                                  "algorithmic_bytes_per_episode_per_layer": round(bytes_all)},
+        "e2e": {"value": round(e2e_v, 3), "unit": "us/attention-call (one layer, one denoise step)",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "note": "bytes per attention call; each denoise step moves L times this"},
+        "gpu_launches": int(n_launch),
         "clocks": clocks,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -463,8 +500,9 @@ def cpu_baseline(workload: str, seed: int, budget_s: float = 12.0) -> dict:
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": round(dt / (n * S) * 1e6, 1), "unit": "us/denoise-step", "cores": _oracle_threads(),
-            "kind": "oracle", "sample": f"{n} full episode(s) of {S} denoise steps, every row and head, fp64 numpy"}
+    return {"value": round(dt / (n * S) * 1e6, 1), "unit": "us/attention-call (one layer, one denoise step)",
+            "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"{n} full episode(s) of {S} denoise steps of one layer, every row and head, fp64 numpy"}
 
 
 def reference(args, world, rank):
@@ -487,7 +525,7 @@ def reference(args, world, rank):
         "impl": "reference",
         "metric": METRIC,
         "value": round(us, 1),
-        "unit": "us/denoise-step",
+        "unit": "us/attention-call (one layer, one denoise step)",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -498,10 +536,12 @@ def reference(args, world, rank):
         "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": WORKLOAD_DESC[args.workload],
-                   "bench_step": f"one denoise episode ({S} steps) of the fp64 oracle on host cores"},
-        "cpu_baseline": {"value": round(us, 1), "unit": "us/denoise-step", "cores": cores, "kind": "oracle",
-                         "sample": f"{args.steps} full episode(s) of {S} denoise steps, every row and head"},
-        "e2e": {"value": round(us, 1), "unit": "us/denoise-step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                   "bench_step": f"one denoise episode ({S} steps) of one layer, fp64 oracle on host cores"},
+        "cpu_baseline": {"value": round(us, 1), "unit": "us/attention-call (one layer, one denoise step)",
+                         "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} full episode(s) of {S} denoise steps of one layer, every row and head"},
+        "e2e": {"value": round(us, 1), "unit": "us/attention-call (one layer, one denoise step)",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
 
@@ -513,6 +553,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=sorted(WORKLOAD_DESC), default="dllm_layer")
+    ap.add_argument("--layers", type=int, default=0, help="attention layers per denoise step (0: workload default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args(argv)

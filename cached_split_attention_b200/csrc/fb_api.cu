@@ -56,6 +56,9 @@ fb_status check_problem(const fb_problem* p) {
     return fail(FB_ERR_INVALID_ARG, "a per-sequence maximum exceeds its total");
   if (p->max_q > p->max_kv_in) return fail(FB_ERR_INVALID_ARG, "max_q exceeds max_kv_in (rows are block positions)");
   if (p->out_splits < 0) return fail(FB_ERR_INVALID_ARG, "out_splits < 0");
+  if (static_cast<int64_t>(p->total_kv_in) * p->num_heads_q >= (int64_t{1} << 31) ||
+      static_cast<int64_t>(p->total_q) * p->num_heads_q >= (int64_t{1} << 31))
+    return fail(FB_ERR_UNSUPPORTED, "tokens x query heads must stay below 2^31");
   if (p->num_seqs > 0 && (!p->cu_seqlens_q || !p->cu_seqlens_kv_out || !p->cu_seqlens_kv_in))
     return fail(FB_ERR_INVALID_ARG, "cu_seqlens arrays must not be NULL");
   return FB_OK;

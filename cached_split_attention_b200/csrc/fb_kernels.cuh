@@ -29,7 +29,7 @@
 // evict-first L2 policy) through a ring of mbarrier-guarded stages.  Warp
 // (wm, wn) owns 16 rows and a 1/WN share of the keys of every stage and runs
 // mma.sync m16n8k16 (bf16 in, fp32 accumulate) with an online softmax in base 2;
-// the WN shares of a row slab are merged through shared memory.
+// each warp hands off its own sub-partial and the merge combines all of them.
 #pragma once
 
 #include <limits>
@@ -43,6 +43,7 @@ constexpr int kBN = 64;        // keys per pipeline stage
 constexpr int kMaxGroup = 32;  // q-heads per kv-head
 constexpr int kMaxSplits = 8;  // CTAs per cluster (portable limit)
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kNegInf = -std::numeric_limits<float>::infinity();
 
 __device__ int g_status;  // first error recorded by any kernel (0 = none)
@@ -102,16 +103,18 @@ __device__ __forceinline__ bool head_recompute(const Params& p, int b, int h) {
   return !reuse;
 }
 
-// Prefix chunks [a, b) of CTA s of S.  The last CTA also runs `in_chunks` block
-// chunks, so it takes fewer prefix chunks; the rest are spread evenly.
+// Prefix chunks [a, b) of CTA s of S.  The last CTA also runs the `in_chunks`
+// block chunks, so it takes fewer prefix chunks; the rest are spread evenly.
 __device__ __forceinline__ void prefix_range(int s, int S, int out_chunks, int in_chunks, int& a, int& b) {
   if (S == 1) {
     a = 0;
     b = out_chunks;
     return;
   }
-  const int per = (out_chunks + in_chunks + S - 1) / S;
-  const int last = min(out_chunks, max(0, per - in_chunks));
+  // the block segment costs its chunks plus about two chunks of hand-off
+  const int in_cost = in_chunks > 0 ? in_chunks + 2 : 0;
+  const int per = (out_chunks + in_cost + S - 1) / S;
+  const int last = min(out_chunks, max(0, per - in_cost));
   const int rest = out_chunks - last;
   if (s == S - 1) {
     a = rest;
@@ -121,6 +124,75 @@ __device__ __forceinline__ void prefix_range(int s, int S, int out_chunks, int i
   const int q = rest / (S - 1), r = rest % (S - 1);
   a = s * q + min(s, r);
   b = a + q + (s < r ? 1 : 0);
+}
+
+// Log-space sum of N normalised partials with base-2 log-normalisers l2[k]
+// (empty partials: -inf):  out = sum_k 2^{l2[k]-m} a[k] / sum_k 2^{l2[k]-m},
+// returning m + log2 sum_k 2^{l2[k]-m} (m = max_k l2[k]); (0, -inf) when every
+// partial is empty.  Hardware ex2 / lg2 / rcp approximations (relative error
+// about 2^-22), well below the bf16 output resolution.
+template <int N>
+__device__ __forceinline__ float lse2_combine(const float (&l2)[N], const float4 (&a)[N], float4& out) {
+  float mx = kNegInf;
+#pragma unroll
+  for (int k = 0; k < N; ++k) mx = fmaxf(mx, l2[k]);
+  out = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mx == kNegInf) return kNegInf;
+  float den = 0.f;
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    if (l2[k] == kNegInf) continue;  // empty partial (its A may be unset)
+    const float w = ex2(l2[k] - mx);
+    den += w;
+    out.x = fmaf(w, a[k].x, out.x);
+    out.y = fmaf(w, a[k].y, out.y);
+    out.z = fmaf(w, a[k].z, out.z);
+    out.w = fmaf(w, a[k].w, out.w);
+  }
+  const float inv = rcp_approx(den);
+  out.x *= inv;
+  out.y *= inv;
+  out.z *= inv;
+  out.w *= inv;
+  return mx + lg2_approx(den);
+}
+
+// Weights of the log-space sum of N partials with base-2 log-normalisers l2[k]:
+// w[k] = 2^{l2[k]-m} / sum_j 2^{l2[j]-m}; returns m + log2 sum_j 2^{l2[j]-m}
+// (m = max l2), or -inf with all weights 0 when every partial is empty.
+template <int N>
+__device__ __forceinline__ float log2_weights(const float (&l2)[N], float* w) {
+  float mx = kNegInf;
+#pragma unroll
+  for (int k = 0; k < N; ++k) mx = fmaxf(mx, l2[k]);
+  if (mx == kNegInf) {
+#pragma unroll
+    for (int k = 0; k < N; ++k) w[k] = 0.f;
+    return kNegInf;
+  }
+  float e[N];
+  float den = 0.f;
+#pragma unroll
+  for (int k = 0; k < N; ++k) {
+    e[k] = l2[k] == kNegInf ? 0.f : ex2(l2[k] - mx);
+    den += e[k];
+  }
+  const float inv = rcp_approx(den);
+#pragma unroll
+  for (int k = 0; k < N; ++k) w[k] = e[k] * inv;
+  return mx + lg2_approx(den);
+}
+
+__device__ __forceinline__ void fma4(float4& acc, float w, const float4& v) {
+  acc.x = fmaf(w, v.x, acc.x);
+  acc.y = fmaf(w, v.y, acc.y);
+  acc.z = fmaf(w, v.z, acc.z);
+  acc.w = fmaf(w, v.w, acc.w);
+}
+
+// Store the folded (natural-log) normaliser of row r of a partial.
+__device__ __forceinline__ void part_l_fold(float* part, int off_l, int r, float lse2) {
+  part[off_l + r] = lse2 == kNegInf ? kNegInf : lse2 * kLn2;
 }
 
 template <int D, int WM, int WN, int STAGES>
@@ -135,20 +207,27 @@ struct Cfg {
   static constexpr int kStageArea = STAGES * kStageBytes;
   static constexpr int kQStride = D + 8;  // padded Q row, elements
   static constexpr int kQBytes = kRows * kQStride * 2;
-  static constexpr int kRegs = D / 2 + 4;  // o, m, l of one lane
-  static constexpr int kScratchBytes = (WN - 1) * WM * 32 * kRegs * 4;
   static constexpr int kPStride = D + 4;  // padded partial row, floats
-  static constexpr int kPartBytes = kRows * kPStride * 4 + kRows * 4;
+  // A partial of the tile is WN sub-partials, one per key share:
+  // A [WN][kRows][kPStride] floats, then L [WN][kRows] floats.
+  static constexpr int kPartL = WN * kRows * kPStride;  // offset of L, floats
+  static constexpr int kPartBytes = (kPartL + WN * kRows) * 4;
   static constexpr int kOffQ = kStageArea;
-  static constexpr int kOffScratch = kOffQ + kQBytes;
-  static constexpr int kOffIn = kOffScratch + kScratchBytes;
+  static constexpr int kOffIn = kOffQ + kQBytes;
   static constexpr int kOffBar = kOffIn + kPartBytes;
   static constexpr int kOffPos = kOffBar + 2 * STAGES * 8;
-  static constexpr int kSmem = 1024 + kOffPos + kRows * 4;
+  // Cached A_out / L_out rows of heads that reuse, copied in while the attention
+  // runs (tiles of up to 32 rows; larger tiles read them from L2 at the merge).
+  static constexpr bool kStageCache = kRows <= 32;
+  static constexpr int kOffCache = (kOffPos + kRows * 4 + 15) / 16 * 16;
+  static constexpr int kCacheBytes = kStageCache ? kRows * kPStride * 4 + kRows * 4 : 0;
+  static constexpr int kSmem = 1024 + kOffCache + kCacheBytes;
   static_assert(kKW % 16 == 0, "keys per warp must be a multiple of 16");
   static_assert(kPartBytes <= kStageArea, "the prefix partial must fit in the stage ring");
-  static_assert(kPartBytes % 16 == 0 && kOffIn % 16 == 0, "16-byte aligned partials");
+  static_assert(kOffIn % 16 == 0 && kOffBar % 8 == 0, "aligned regions");
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(32 % (D / 4) == 0 && kThreads % 32 == 0, "a row's float4 items share one warp");
+  static_assert(kRows * (kMaxSplits + WN + 6) * 4 <= kQBytes, "per-row merge weights fit in the Q tile");
 };
 
 // Byte offset of (key row kr, column dd) inside a stage tile written by TMA with
@@ -270,12 +349,12 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
   __nv_bfloat16* q_s = reinterpret_cast<__nv_bfloat16*>(smem + C::kOffQ);
-  float* scratch = reinterpret_cast<float*>(smem + C::kOffScratch);
-  float* in_part = reinterpret_cast<float*>(smem + C::kOffIn);  // block partial: A [TR][kPStride], L [TR]
+  float* in_part = reinterpret_cast<float*>(smem + C::kOffIn);  // block partial
   float* out_part = reinterpret_cast<float*>(stages);            // prefix partial, after the ring drains
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + STAGES;
-  int* s_pos = reinterpret_cast<int*>(smem + C::kOffPos);  // block position of each tile row (-1: bad)
+  int* s_pos = reinterpret_cast<int*>(smem + C::kOffPos);  // block position of each tile row (-1: none)
+  float* cache_s = reinterpret_cast<float*>(smem + C::kOffCache);  // staged cache rows (kStageCache)
   __shared__ uint8_t s_rec[kMaxGroup];
   __shared__ int s_flag;
 
@@ -301,6 +380,17 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   const int in0 = p.cu_in[b];
   const int n_in = p.cu_in[b + 1] - in0;
   if (tid < g) s_rec[tid] = head_recompute(p, b, hk * g + tid) ? 1 : 0;
+  // The cache-state epilogue only runs when some entry is still empty (valid = 0).
+  int invalid = 0;
+  if (p.update_state) {
+    const int total = p.num_seqs * p.hq;
+    if (total > 8 * C::kThreads) {
+      invalid = 1;
+    } else {
+      for (int i = tid; i < total; i += C::kThreads) invalid |= p.valid[i] == 0;
+    }
+  }
+  const bool need_state = __syncthreads_or(invalid) != 0;
   const bool ranges_ok = q0 >= 0 && n_q >= 0 && q0 + n_q <= p.total_q && out0 >= 0 && n_out >= 0 &&
                          out0 + n_out <= p.total_out && in0 >= 0 && n_in >= 0 && in0 + n_in <= p.total_in &&
                          n_q <= n_in;
@@ -308,7 +398,6 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   const int rows = ranges_ok ? n_q * g : 0;
   const int row0 = t * TR;
   const int nrows = max(0, min(TR, rows - row0));
-  __syncthreads();
   bool any_rec = false;
   for (int j = 0; j < g; ++j) any_rec |= (s_rec[j] != 0);
 
@@ -322,14 +411,17 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   const bool has_out = do_out && (pb > pa || (out_chunks == 0 && split == 0));
   const bool cluster_mode = S > 1 && do_out;  // uniform over the cluster
   const bool active = nrows > 0;               // uniform over the cluster
-  // The block segment (if any) runs first; its partial goes to a dedicated
-  // region.  The prefix segment runs last, so its partial can reuse the ring.
+  // The block segment (if any) runs first into a region of its own; the prefix
+  // segment runs last, so its partial can reuse the drained ring.
   const int nA = has_in ? in_chunks : 0;
   const int nB = has_out ? pb - pa : 0;
   const int n_local = nA + nB;
-  // Which CTA merges which rows: all CTAs of a cluster share the rows; otherwise
-  // the CTA that holds every partial merges them all.
+  // Merging: all CTAs of a cluster share the rows; otherwise the CTA that holds
+  // every partial merges all of them.
   const bool merger = cluster_mode || has_in || (S == 1 && has_out);
+
+  // decisions of this group's heads (written once per (b, kv-head))
+  if (p.decision_out && t == 0 && split == S - 1 && tid < g) p.decision_out[b * p.hq + hk * g + tid] = s_rec[tid];
 
   if (active && (has_in || has_out || cluster_mode)) {
     // -------------------------------------------------------- Q rows first
@@ -349,17 +441,17 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
                                                 c * 8);
       }
     }
-    for (int r = tid; r < TR; r += C::kThreads) {
-      int pos = -1;
+    // block positions of the tile rows (also before the flood)
+    constexpr int kPosPer = (TR + C::kThreads - 1) / C::kThreads;
+    int posv[kPosPer];
+#pragma unroll
+    for (int k = 0; k < kPosPer; ++k) {
+      const int r = tid + k * C::kThreads;
+      posv[k] = -1;
       if (r < nrows) {
         const int it = (row0 + r) / g;
-        pos = p.q_rows ? p.q_rows[q0 + it] : it;
-        if (pos < 0 || pos >= n_in) {
-          record_status(kDevBadIndex);
-          pos = -1;
-        }
+        posv[k] = p.q_rows ? p.q_rows[q0 + it] : it;
       }
-      s_pos[r] = pos;
     }
     // -------------------------------------------------------- TMA ring
     if (tid == 0) {
@@ -390,17 +482,32 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
       pol = l2_policy_evict_first();
       for (int c = 0; c < min(STAGES, n_local); ++c) issue(c);
     }
-    // cached rows this CTA will merge with: bring them into L2 early
-    if (merger && p.fused) {
-      for (int r = tid; r < nrows; r += C::kThreads) {
+    // cached rows this CTA merges with go to L2 while the attention runs
+#pragma unroll
+    for (int k = 0; k < kPosPer; ++k) {
+      const int r = tid + k * C::kThreads;
+      if (r >= TR) continue;
+      int pos = posv[k];
+      if (r < nrows) {
         const int rho = row0 + r;
-        if (s_rec[rho % g]) continue;
-        const int it = rho / g;
-        const int pos = p.q_rows ? p.q_rows[q0 + it] : it;
-        if (pos >= 0 && pos < n_in)
-          prefetch_l2(p.cache_a + (static_cast<size_t>(in0 + pos) * p.hq + hk * g + rho % g) * D, D * 4);
+        if (pos < 0 || pos >= n_in) {
+          record_status(kDevBadIndex);
+          pos = -1;
+        } else if (merger && p.fused && !(do_out && s_rec[rho % g])) {
+          const size_t ce = static_cast<size_t>(in0 + pos) * p.hq + hk * g + rho % g;
+          if constexpr (C::kStageCache) {
+            for (int c = 0; c < D / 4; ++c)
+              cp_async_16(cache_s + r * C::kPStride + c * 4, p.cache_a + ce * D + c * 4);
+            cp_async_4(cache_s + TR * C::kPStride + r, p.cache_l + ce);
+          } else {
+            prefetch_l2(p.cache_a + ce * D, D * 4);
+            prefetch_l2_line(p.cache_l + ce);
+          }
+        }
       }
+      s_pos[r] = pos;
     }
+    cp_async_commit();
 #pragma unroll
     for (int k = 0; k < kQPer; ++k) {
       const int v = tid + k * C::kThreads;
@@ -466,71 +573,30 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
         }
       }
     };
-
-    // Close a segment: merge the WN key-shares of every row slab and store the
-    // normalised partial (A, L = ln Z) of the tile in `dst` ([TR][kPStride], then [TR]).
+    // Each warp stores its own normalised sub-partial (A, L = ln Z) of its 16 rows
+    // and key share into `dst` ([WN][TR][kPStride], then [WN][TR]).
     auto close = [&](float* dst) {
-      float l_tot[2];
-      l_tot[0] = quad_sum(acc.l[0]);
-      l_tot[1] = quad_sum(acc.l[1]);
-      if constexpr (WN > 1) {
-        __syncthreads();
-        if (wn > 0) {
-          float* mine = scratch + ((wn - 1) * WM + wm) * C::kRegs * 32;
+      float z[2];
+      z[0] = quad_sum(acc.l[0]);
+      z[1] = quad_sum(acc.l[1]);
 #pragma unroll
-          for (int n = 0; n < D / 8; ++n)
+      for (int i = 0; i < 2; ++i) {
+        const int r = 16 * wm + (lane >> 2) + 8 * i;
+        const float inv = z[i] > 0.f ? 1.f / z[i] : 0.f;
+        float* row = dst + (wn * TR + r) * C::kPStride;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) mine[(n * 4 + e) * 32 + lane] = acc.o[n][e];
-          mine[(D / 2 + 0) * 32 + lane] = acc.m[0];
-          mine[(D / 2 + 1) * 32 + lane] = acc.m[1];
-          mine[(D / 2 + 2) * 32 + lane] = l_tot[0];
-          mine[(D / 2 + 3) * 32 + lane] = l_tot[1];
-        }
-        __syncthreads();
-        if (wn == 0) {
-#pragma unroll 1
-          for (int w2 = 1; w2 < WN; ++w2) {
-            const float* th = scratch + ((w2 - 1) * WM + wm) * C::kRegs * 32;
-            float a1[2], a2[2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const float m2 = th[(D / 2 + i) * 32 + lane];
-              const float l2 = th[(D / 2 + 2 + i) * 32 + lane];
-              const float mn = fmaxf(acc.m[i], m2);
-              const float ms = mn == kNegInf ? 0.f : mn;
-              a1[i] = ex2(acc.m[i] - ms);
-              a2[i] = ex2(m2 - ms);
-              l_tot[i] = l_tot[i] * a1[i] + l2 * a2[i];
-              acc.m[i] = mn;
-            }
-#pragma unroll
-            for (int n = 0; n < D / 8; ++n) {
-              acc.o[n][0] = acc.o[n][0] * a1[0] + th[(n * 4 + 0) * 32 + lane] * a2[0];
-              acc.o[n][1] = acc.o[n][1] * a1[0] + th[(n * 4 + 1) * 32 + lane] * a2[0];
-              acc.o[n][2] = acc.o[n][2] * a1[1] + th[(n * 4 + 2) * 32 + lane] * a2[1];
-              acc.o[n][3] = acc.o[n][3] * a1[1] + th[(n * 4 + 3) * 32 + lane] * a2[1];
-            }
-          }
-        }
-      } else {
-        __syncthreads();  // the ring may be reused as the destination
-      }
-      if (wn == 0) {
-        float* dl = dst + TR * C::kPStride;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int r = 16 * wm + (lane >> 2) + 8 * i;
-          const float z = l_tot[i];
-          const float inv = z > 0.f ? 1.f / z : 0.f;
-#pragma unroll
-          for (int n = 0; n < D / 8; ++n)
-            *reinterpret_cast<float2*>(dst + r * C::kPStride + n * 8 + 2 * (lane & 3)) =
-                make_float2(acc.o[n][2 * i] * inv, acc.o[n][2 * i + 1] * inv);
-          if ((lane & 3) == 0) dl[r] = z > 0.f ? (acc.m[i] + log2f(z)) * kLn2 : kNegInf;
-        }
+        for (int n = 0; n < D / 8; ++n)
+          *reinterpret_cast<float2*>(row + n * 8 + 2 * (lane & 3)) =
+              make_float2(acc.o[n][2 * i] * inv, acc.o[n][2 * i + 1] * inv);
+        if ((lane & 3) == 0) dst[C::kPartL + wn * TR + r] = z[i] > 0.f ? (acc.m[i] + log2f(z[i])) * kLn2 : kNegInf;
       }
       acc.reset();
-      __syncthreads();  // the partial is complete before any warp reads it
+    };
+    auto drain = [&]() {  // copies issued but never consumed (after a timeout) land first
+      if (tid == 0 && !ok) {
+        for (int c = max(0, issued - STAGES); c < issued; ++c)
+          if (!mbar_wait(&full[c % STAGES], (c / STAGES) & 1)) record_status(kDevTimeout);
+      }
     };
 
     // -------------------------------------------------------- the two segments
@@ -540,137 +606,211 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
     }
     if (has_out) {
       run(nA, n_local);
-      // every issued copy has landed before the ring is reused
-      if (tid == 0 && !ok) {
-        for (int c = max(0, issued - STAGES); c < issued; ++c)
-          if (!mbar_wait(&full[c % STAGES], (c / STAGES) & 1)) record_status(kDevTimeout);
-      }
+      drain();
+      __syncthreads();  // every warp is done with the ring before it holds the partial
       close(out_part);
-    } else if (tid == 0 && !ok) {
-      for (int c = max(0, issued - STAGES); c < issued; ++c)
-        if (!mbar_wait(&full[c % STAGES], (c / STAGES) & 1)) record_status(kDevTimeout);
+    } else {
+      drain();
     }
 
     // -------------------------------------------------------- merge
-    if (cluster_mode) cluster_sync();
+    constexpr int kC4 = D / 4;  // float4 columns of a row
+    // Step 1, in place: each partial this CTA holds becomes one partial per row
+    // (its WN key-share sub-partials combined into sub-partial 0).
+    __syncthreads();
+    auto fold = [&](float* part) {
+      for (int item = tid; item < nrows * kC4; item += C::kThreads) {
+        const int r = item / kC4;
+        const int c4 = (item % kC4) * 4;
+        float l2[WN];
+        float4 a[WN];
+#pragma unroll
+        for (int w = 0; w < WN; ++w) {
+          l2[w] = part[C::kPartL + w * TR + r] * kLog2e;
+          a[w] = *reinterpret_cast<const float4*>(part + (w * TR + r) * C::kPStride + c4);
+        }
+        float4 o;
+        const float lse2 = lse2_combine<WN>(l2, a, o);
+        // The items of a row are consecutive lanes of one warp (kC4 divides 32):
+        // they have all read the row's L values before one of them rewrites them.
+        __syncwarp(__activemask());
+        *reinterpret_cast<float4*>(part + r * C::kPStride + c4) = o;
+        if (c4 == 0) part_l_fold(part, C::kPartL, r, lse2);
+      }
+    };
+    if (WN > 1 && cluster_mode) {  // cluster merges read one partial per CTA
+      if (has_in) fold(in_part);
+      if (has_out) fold(out_part);
+    }
+    cp_async_wait_all();
+    if (cluster_mode) {
+      cluster_sync();
+    } else {
+      __syncthreads();
+    }
     if (merger) {
       const int rp = cluster_mode ? (nrows + S - 1) / S : nrows;
       const int r_lo = cluster_mode ? split * rp : 0;
       const int r_hi = min(nrows, r_lo + rp);
-      const uint32_t out_l = smem_u32(out_part);
-      const uint32_t in_l = smem_u32(in_part);
-      constexpr int kC4 = D / 4;  // float4 columns of a row
-      // owners of prefix partials (same schedule on every CTA of the cluster)
-      uint32_t owners = 0;
+      const uint32_t out_a = smem_u32(out_part);
+      const uint32_t in_a = smem_u32(in_part);
+      uint32_t owners = 0;  // CTAs holding a prefix partial
       for (int s2 = 0; s2 < S; ++s2) {
         int a0, a1;
         prefix_range(s2, S, out_chunks, in_chunks, a0, a1);
         if (a1 > a0) owners |= 1u << s2;
       }
-      for (int item = tid; item < (r_hi - r_lo) * kC4; item += C::kThreads) {
-        const int r = r_lo + item / kC4;
-        const int c4 = (item % kC4) * 4;
+      auto ld_f = [&](uint32_t base, int rank, int f) -> float {
+        const uint32_t ad = base + f * 4;
+        return cluster_mode ? ld_dsmem_f32(dsmem_addr(ad, rank)) : ld_shared_f32(ad);
+      };
+      auto ld_f4 = [&](uint32_t base, int rank, int f) -> float4 {
+        const uint32_t ad = base + f * 4;
+        return cluster_mode ? ld_dsmem_f4(dsmem_addr(ad, rank)) : ld_shared_f4(ad);
+      };
+      const int n_items = (r_hi - r_lo) * kC4;
+      // Entries of a row: prefix entry k is the folded partial of CTA k (cluster
+      // mode) or this CTA's key-share sub-partial k; block entry w likewise
+      // (folded partial of the last CTA in cluster mode, sub-partial w otherwise).
+      constexpr int kOutE = kMaxSplits;
+      constexpr int kInE = WN;
+      const int n_out_e = cluster_mode ? S : WN;
+      const int n_in_e = cluster_mode ? 1 : WN;
+      // Phase W, one thread per row: every weight of the row and where it goes.
+      // Row slot (kWt floats): [0,kOutE) prefix weights, [kOutE,+kInE) block weights
+      // (already scaled by the block's share of A_full), then wo (A_out's share of
+      // A_full), L_out, L_full (or L_in), kind, cache entry, output entry.
+      float* wt = reinterpret_cast<float*>(q_s);  // the Q tile is dead by now
+      constexpr int kWt = kOutE + kInE + 6;
+      for (int r = r_lo + tid; r < r_hi; r += C::kThreads) {
+        float* wr = wt + (r - r_lo) * kWt;
         const int pos = s_pos[r];
-        if (pos < 0) continue;
         const int rho = row0 + r;
         const int j = rho % g;
-        const int h = hk * g + j;
-        const size_t ce = static_cast<size_t>(in0 + pos) * p.hq + h;
-        const bool rec = s_rec[j] != 0;
-        float4 ao = make_float4(0.f, 0.f, 0.f, 0.f);
-        float lo = kNegInf;
-        if (do_out && rec) {
-          // prefix partials of the owners: all loads first, then the log-space sum
-          float ls[kMaxSplits];
-          float4 as[kMaxSplits];
+        float kind = 0.f;
+        float lo2 = kNegInf, li2 = kNegInf;
+        if (pos >= 0) {
+          const int ce = (in0 + pos) * p.hq + hk * g + j;
+          wr[kOutE + kInE + 4] = __int_as_float(ce);
+          wr[kOutE + kInE + 5] = __int_as_float((q0 + rho / g) * p.hq + hk * g + j);
+          if (do_out && s_rec[j]) {
+            float l2[kOutE];
 #pragma unroll
-          for (int s2 = 0; s2 < kMaxSplits; ++s2) {
-            ls[s2] = kNegInf;
-            if (s2 < S && (owners >> s2 & 1u)) {
-              const uint32_t rank = cluster_mode ? s2 : split;
-              const uint32_t lb = out_l + (TR * C::kPStride + r) * 4;
-              const uint32_t ab = out_l + (r * C::kPStride + c4) * 4;
-              ls[s2] = cluster_mode ? ld_dsmem_f32(dsmem_addr(lb, rank)) : out_part[TR * C::kPStride + r];
-              as[s2] = cluster_mode ? ld_dsmem_f4(dsmem_addr(ab, rank))
-                                    : *reinterpret_cast<const float4*>(out_part + r * C::kPStride + c4);
+            for (int k = 0; k < kOutE; ++k) {
+              l2[k] = kNegInf;
+              if (k < n_out_e && (owners >> (cluster_mode ? k : 0) & 1u))
+                l2[k] = (cluster_mode ? ld_f(out_a, k, C::kPartL + r) : out_part[C::kPartL + k * TR + r]) * kLog2e;
             }
-          }
-          float mx = kNegInf;
-#pragma unroll
-          for (int s2 = 0; s2 < kMaxSplits; ++s2) mx = fmaxf(mx, ls[s2]);
-          if (mx != kNegInf) {
-            float den = 0.f;
-#pragma unroll
-            for (int s2 = 0; s2 < kMaxSplits; ++s2) {
-              if (ls[s2] == kNegInf) continue;
-              const float w = expf(ls[s2] - mx);
-              den += w;
-              ao.x += w * as[s2].x;
-              ao.y += w * as[s2].y;
-              ao.z += w * as[s2].z;
-              ao.w += w * as[s2].w;
-            }
-            const float inv = 1.f / den;
-            ao.x *= inv;
-            ao.y *= inv;
-            ao.z *= inv;
-            ao.w *= inv;
-            lo = mx + logf(den);
-          }
-          *reinterpret_cast<float4*>(p.cache_a + ce * D + c4) = ao;
-          if (c4 == 0) p.cache_l[ce] = lo;
-        } else if (p.fused) {
-          ao = *reinterpret_cast<const float4*>(p.cache_a + ce * D + c4);
-          lo = p.cache_l[ce];
-        }
-        if (p.do_in) {
-          // the block partial lives in the last CTA of the cluster
-          const uint32_t rank = S - 1;
-          const float li = cluster_mode ? ld_dsmem_f32(dsmem_addr(in_l + (TR * C::kPStride + r) * 4, rank))
-                                        : in_part[TR * C::kPStride + r];
-          const float4 ai = cluster_mode ? ld_dsmem_f4(dsmem_addr(in_l + (r * C::kPStride + c4) * 4, rank))
-                                         : *reinterpret_cast<const float4*>(in_part + r * C::kPStride + c4);
-          const size_t fe = static_cast<size_t>(q0 + rho / g) * p.hq + h;
-          if (!p.fused) {
-            *reinterpret_cast<float4*>(p.a_in + fe * D + c4) = ai;
-            if (c4 == 0) p.l_in[fe] = li;
+            lo2 = log2_weights<kOutE>(l2, wr);
+            kind = 1.f;
+          } else if (p.fused) {
+            lo2 = (C::kStageCache ? cache_s[TR * C::kPStride + r] : p.cache_l[ce]) * kLog2e;
+            kind = 2.f;
           } else {
-            const float mx = fmaxf(lo, li);
-            float wo = 0.f, wi = 0.f, lf = kNegInf;
-            if (mx != kNegInf) {
-              wo = lo == kNegInf ? 0.f : expf(lo - mx);
-              wi = li == kNegInf ? 0.f : expf(li - mx);
-              const float den = wo + wi;
-              lf = mx + logf(den);
-              wo /= den;
-              wi /= den;
+            kind = 3.f;  // block pass alone
+          }
+          if (p.do_in) {
+            float l2[kInE];
+#pragma unroll
+            for (int w = 0; w < kInE; ++w) {
+              l2[w] = kNegInf;
+              if (w < n_in_e)
+                l2[w] = (cluster_mode ? ld_f(in_a, S - 1, C::kPartL + r) : in_part[C::kPartL + w * TR + r]) * kLog2e;
             }
-            __nv_bfloat16* dst = p.a_full + fe * D + c4;
-            *reinterpret_cast<__nv_bfloat162*>(dst) =
-                __floats2bfloat162_rn(wo * ao.x + wi * ai.x, wo * ao.y + wi * ai.y);
-            *reinterpret_cast<__nv_bfloat162*>(dst + 2) =
-                __floats2bfloat162_rn(wo * ao.z + wi * ai.z, wo * ao.w + wi * ai.w);
-            if (c4 == 0 && p.l_full) p.l_full[fe] = lf;
+            li2 = log2_weights<kInE>(l2, wr + kOutE);
           }
         }
+        float wo = 1.f, lf2 = li2;
+        if (p.fused && pos >= 0) {
+          const float m2 = fmaxf(lo2, li2);
+          wo = 0.f;
+          float wi = 0.f;
+          lf2 = kNegInf;
+          if (m2 != kNegInf) {
+            wo = lo2 == kNegInf ? 0.f : ex2(lo2 - m2);
+            wi = li2 == kNegInf ? 0.f : ex2(li2 - m2);
+            const float inv = rcp_approx(wo + wi);
+            lf2 = m2 + lg2_approx(wo + wi);
+            wo *= inv;
+            wi *= inv;
+          }
+#pragma unroll
+          for (int w = 0; w < kInE; ++w) wr[kOutE + w] *= wi;
+        }
+        wr[kOutE + kInE + 0] = wo;
+        wr[kOutE + kInE + 1] = lo2 == kNegInf ? kNegInf : lo2 * kLn2;
+        wr[kOutE + kInE + 2] = lf2 == kNegInf ? kNegInf : lf2 * kLn2;
+        wr[kOutE + kInE + 3] = kind;
+      }
+      __syncthreads();
+      // Phase C, (row, 4 columns) items: loads and multiply-adds only.
+      for (int item = tid; item < n_items; item += C::kThreads) {
+        const int r = r_lo + item / kC4;
+        const int c4 = (item % kC4) * 4;
+        const float* wr = wt + (r - r_lo) * kWt;
+        const int kind = static_cast<int>(wr[kOutE + kInE + 3]);
+        if (kind == 0) continue;
+        const size_t ce = static_cast<unsigned>(__float_as_int(wr[kOutE + kInE + 4]));
+        const size_t fe = static_cast<unsigned>(__float_as_int(wr[kOutE + kInE + 5]));
+        float4 ao = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (kind == 1) {
+          float4 v[kOutE];
+#pragma unroll
+          for (int k = 0; k < kOutE; ++k) {
+            if (wr[k] == 0.f) continue;
+            v[k] = cluster_mode ? ld_f4(out_a, k, r * C::kPStride + c4)
+                                : *reinterpret_cast<const float4*>(out_part + (k * TR + r) * C::kPStride + c4);
+          }
+#pragma unroll
+          for (int k = 0; k < kOutE; ++k)
+            if (wr[k] != 0.f) fma4(ao, wr[k], v[k]);
+          *reinterpret_cast<float4*>(p.cache_a + ce * D + c4) = ao;
+          if (c4 == 0) p.cache_l[ce] = wr[kOutE + kInE + 1];
+        } else if (kind == 2) {
+          ao = C::kStageCache ? *reinterpret_cast<const float4*>(cache_s + r * C::kPStride + c4)
+                              : *reinterpret_cast<const float4*>(p.cache_a + ce * D + c4);
+        }
+        if (!p.do_in) continue;
+        float4 ai = make_float4(0.f, 0.f, 0.f, 0.f);
+        {
+          float4 v[kInE];
+#pragma unroll
+          for (int w = 0; w < kInE; ++w) {
+            if (w >= n_in_e) continue;
+            v[w] = cluster_mode ? ld_f4(in_a, S - 1, r * C::kPStride + c4)
+                                : *reinterpret_cast<const float4*>(in_part + (w * TR + r) * C::kPStride + c4);
+          }
+#pragma unroll
+          for (int w = 0; w < kInE; ++w)
+            if (w < n_in_e) fma4(ai, wr[kOutE + w], v[w]);
+        }
+        if (!p.fused) {
+          *reinterpret_cast<float4*>(p.a_in + fe * D + c4) = ai;
+          if (c4 == 0) p.l_in[fe] = wr[kOutE + kInE + 2];
+          continue;
+        }
+        const float wo = wr[kOutE + kInE + 0];
+        __nv_bfloat16* dst = p.a_full + fe * D + c4;
+        *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(fmaf(wo, ao.x, ai.x), fmaf(wo, ao.y, ai.y));
+        *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(fmaf(wo, ao.z, ai.z), fmaf(wo, ao.w, ai.w));
+        if (c4 == 0 && p.l_full) p.l_full[fe] = wr[kOutE + kInE + 2];
       }
     }
     if (cluster_mode) cluster_sync();  // no CTA leaves while its partials may still be read
   }
 
-  // ------------------------------------------------------------ grid epilogue
-  if (p.update_state) {
+  // ------------------------------------------------------------ cache-state epilogue
+  // Heads that recompute become valid.  Every CTA has read `valid` by now; the
+  // last one to arrive writes it (no CTA waits).
+  if (need_state) {
     __syncthreads();
     if (tid == 0) s_flag = (atomicAdd(p.grid_ctr, 1) == static_cast<int>(gridDim.x) - 1) ? 1 : 0;
     __syncthreads();
     if (s_flag) {
       __threadfence();
       const int total = p.num_seqs * p.hq;
-      for (int idx = tid; idx < total; idx += C::kThreads) {
-        const bool rec = head_recompute(p, idx / p.hq, idx % p.hq);
-        if (p.decision_out) p.decision_out[idx] = rec ? 1 : 0;
-        if (rec) p.valid[idx] = 1;
-      }
+      for (int idx = tid; idx < total; idx += C::kThreads)
+        if (head_recompute(p, idx / p.hq, idx % p.hq)) p.valid[idx] = 1;
       if (tid == 0) *p.grid_ctr = 0;
     }
   }
