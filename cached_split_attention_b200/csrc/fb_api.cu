@@ -81,7 +81,7 @@ fb_status check_ptr(const void* ptr, const char* name, bool needed) {
 
 struct Plan {
   int d = 0, g = 0, wm = 0, tr = 0, tiles = 0, n_groups = 0, splits = 1, threads = 0, smem = 0;
-  size_t off_grid_ctr = 0, off_cos = 0, off_in_a = 0, off_in_l = 0, bytes = 0;
+  size_t off_grid_ctr = 0, off_cos = 0, bytes = 0;
 };
 
 int device_sms() {
@@ -165,10 +165,6 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only) {
   off = align_up(off + sizeof(int), 256);
   pl.off_cos = off;
   off = align_up(off + sizeof(float) * std::max(1, p->num_seqs * p->num_heads_q), 256);
-  pl.off_in_a = off;
-  off = align_up(off + sizeof(float) * static_cast<size_t>(pl.n_groups) * pl.tr * pl.d, 256);
-  pl.off_in_l = off;
-  off = align_up(off + sizeof(float) * static_cast<size_t>(pl.n_groups) * pl.tr, 256);
   pl.bytes = off;
   return pl;
 }
@@ -289,8 +285,6 @@ void fill_workspace(const Plan& pl, void* ws, fb::Params& prm) {
   char* base = static_cast<char*>(ws);
   prm.grid_ctr = reinterpret_cast<int*>(base + pl.off_grid_ctr);
   prm.cos = reinterpret_cast<const float*>(base + pl.off_cos);
-  prm.ws_in_a = reinterpret_cast<float*>(base + pl.off_in_a);
-  prm.ws_in_l = reinterpret_cast<float*>(base + pl.off_in_l);
 }
 
 }  // namespace

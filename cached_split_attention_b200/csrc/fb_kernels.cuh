@@ -84,9 +84,7 @@ struct alignas(64) Params {
   float* a_in;
   float* l_in;
   // workspace
-  float* ws_in_a;  // [groups][TR][D] block partial of a group in cluster mode
-  float* ws_in_l;  // [groups][TR]
-  int* grid_ctr;
+  int* grid_ctr;  // completion counter of the cache-state epilogue (zero between calls)
 };
 
 // Reuse decision of (b, h); see fb_step in flashblock.h.

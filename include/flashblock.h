@@ -118,10 +118,9 @@ const char* fb_last_error(void);
 int32_t fb_version(void);
 
 /*
- * Bytes of workspace that fb_out_attn / fb_step / fb_head_similarity need for
- * this problem (split partials, completion counters, similarity scores).  Pure
- * host computation: plans for the current device's SM count, or for 148 SMs when
- * no device is visible.
+ * Bytes of workspace that fb_out_attn / fb_step need for this problem (a
+ * completion counter and the per-head similarity scores; partials stay on chip).
+ * Pure host computation.
  */
 fb_status fb_workspace_size(const fb_problem* problem, size_t* bytes);
 

@@ -79,10 +79,13 @@ def test_host_validation_without_gpu():
     assert B._lib.fb_merge(-1, 4, 16, 16, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG
 
 
-def test_workspace_size_grows_with_splits():
+def test_workspace_size_is_counter_plus_scores():
+    """The workspace holds a completion counter (256-byte slot) and one fp32
+    similarity score per (sequence, q-head); partials stay on chip."""
     _built()
     from cached_split_attention_b200 import binding as B
-    n1, n8 = ctypes.c_size_t(), ctypes.c_size_t()
-    B._lib.fb_workspace_size(ctypes.byref(_problem(B, out_splits=1)), ctypes.byref(n1))
-    B._lib.fb_workspace_size(ctypes.byref(_problem(B, out_splits=8)), ctypes.byref(n8))
-    assert n8.value > n1.value
+    for seqs, hq, expect in [(1, 32, 256 + 256), (8, 32, 256 + 1024), (3, 40, 256 + 512)]:
+        n = ctypes.c_size_t()
+        prob = _problem(B, num_seqs=seqs, num_heads_q=hq, num_heads_kv=hq, out_splits=4)
+        assert B._lib.fb_workspace_size(ctypes.byref(prob), ctypes.byref(n)) == B.OK
+        assert n.value == expect, (seqs, hq, n.value)
