@@ -71,6 +71,9 @@ def _load():
         "fb_cache_invalidate": (st, [P, ctypes.POINTER(FbCache), vp]),
         "fb_release_cache": (st, []),
         "fb_device_status": (st, [ctypes.POINTER(ctypes.c_int32), vp]),
+        "fb_step_noalloc": (st, [P, ctypes.POINTER(FbParams), ctypes.POINTER(FbCache), vp, vp, vp, vp, vp, vp, vp,
+                                 vp, vp, vp, vp]),
+        "fb_noalloc_last_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)  # AttributeError (loud) if the ABI is incomplete
@@ -200,6 +203,18 @@ def step(problem: DeviceProblem, prm: FbParams, cache: Cache, q, k_in, v_in, k_o
     _check(_lib.fb_step(problem.ref, ctypes.byref(prm), cache.ref, _ptr(q), _ptr(k_in), _ptr(v_in), _ptr(k_out),
                         _ptr(v_out), _ptr(n_updated), _ptr(head_reuse_in), _ptr(a_full), _ptr(l_full),
                         _ptr(decision_out), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def step_noalloc(problem: DeviceProblem, prm: FbParams, cache: Cache, q, k_in, v_in, k_out, v_out, n_updated,
+                 a_full, l_full=None, head_reuse_in=None, decision_out=None, stream=None):
+    """fb_step without a workspace: for callers that cannot allocate device memory,
+    the library uses its own built-in scratch (see fb_step_noalloc in flashblock.h)."""
+    status = _lib.fb_step_noalloc(problem.ref, ctypes.byref(prm), cache.ref, _ptr(q), _ptr(k_in), _ptr(v_in),
+                                  _ptr(k_out), _ptr(v_out), _ptr(n_updated), _ptr(head_reuse_in), _ptr(a_full),
+                                  _ptr(l_full), _ptr(decision_out), _stream(stream))
+    if status != OK:
+        msg = _lib.fb_noalloc_last_error().decode() or last_error()
+        raise FlashBlockError(status, msg)
 
 
 def cache_invalidate(problem: DeviceProblem, cache: Cache, stream=None):

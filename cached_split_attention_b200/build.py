@@ -2,7 +2,7 @@
 
     python -m cached_split_attention_b200.build [--force] [--verbose]
 
-The library is one translation unit (csrc/fb_api.cu includes the kernels);
+The library is csrc/*.cu (fb_api.cu includes the kernels);
 cudart is linked statically, the driver API is reached through
 cudaGetDriverEntryPointByVersion, so the .so needs only libcuda at run time.
 """
@@ -48,8 +48,8 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and up_to_date():
         return LIB
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, *extra,
-           os.path.join(CSRC, "fb_api.cu"), "-o", LIB + ".tmp"]
+    units = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, *extra, *units, "-o", LIB + ".tmp"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)

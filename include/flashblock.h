@@ -205,6 +205,32 @@ fb_status fb_release_cache(void);
  * of bounds. */
 fb_status fb_device_status(int32_t* code, fb_stream_t stream);
 
+/*
+ * fb_step without a workspace argument, for callers that cannot allocate device
+ * memory (a framework allocator owns all of it, a plugin must not allocate, or an
+ * allocation inside the step loop is not acceptable).  The pages describe no such
+ * call; it exists only for these integrations.
+ *
+ * Arguments and results are those of fb_step.  Instead of a caller workspace the
+ * call uses a scratch array built into the library: 64 KiB of device memory that
+ * every GPU loading the library holds until the process exits.  It covers
+ * num_seqs x num_heads_q up to 16320; larger problems return FB_ERR_UNSUPPORTED
+ * (message in fb_noalloc_last_error()) -- use fb_step with a workspace for them.
+ * No call allocates: the first call on a device resolves the scratch address
+ * (cudaGetSymbolAddress), so make that first call before capturing a stream.
+ * Every call on a device shares the one array, which keeps the last call's
+ * contents (the call clears the part that must start at zero): calls that could
+ * overlap on the GPU race and must be ordered, e.g. issued on one stream.
+ * Errors of argument checking are reported through fb_last_error().
+ */
+fb_status fb_step_noalloc(const fb_problem* problem, const fb_params* params, const fb_cache* cache,
+                          const fb_bf16* q, const fb_bf16* k_in, const fb_bf16* v_in, const fb_bf16* k_out,
+                          const fb_bf16* v_out, const int32_t* n_updated, const uint8_t* head_reuse_in,
+                          fb_bf16* a_full, float* l_full, uint8_t* decision_out, fb_stream_t stream);
+
+/* Message of the last fb_step_noalloc failure that is not an argument error. */
+const char* fb_noalloc_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif
