@@ -162,13 +162,15 @@ def run_policy(workload, sample: Optional[Sequence[Tuple[int, int]]] = None,
             rs = rs_all if rows is None else np.asarray([r for r in rows if r0 <= r < r1], dtype=np.int64)
             if len(rs):
                 o0, o1 = int(p.cu_seqlens_kv_out[b]), int(p.cu_seqlens_kv_out[b + 1])
-                for h in heads:
-                    hk = h // g
+                for hk in sorted(set(h // g for h in heads)):
                     kk = bf16_to_f64(workload.k_out[o0:o1, hk])
                     vv = bf16_to_f64(workload.v_out[o0:o1, hk])
-                    a, l = attend(q[rs, h], kk, vv, p.softmax_scale)
-                    cache.a_out[crow[rs], h] = a
-                    cache.l_out[crow[rs], h] = l
+                    for h in heads:
+                        if h // g != hk:
+                            continue
+                        a, l = attend(q[rs, h], kk, vv, p.softmax_scale)
+                        cache.a_out[crow[rs], h] = a
+                        cache.l_out[crow[rs], h] = l
             for h in heads:
                 cache.q_ref[crow[rs_all], h] = q[rs_all, h]
                 cache.valid[b, h] = True
