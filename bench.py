@@ -312,6 +312,19 @@ def _elapsed_us(ev):
     return np.array([[e0.elapsed_time(e1) * 1e3 for e0, e1 in row] for row in ev])
 
 
+def kernel_source_digest() -> str:
+    """sha256 over the CUDA sources of the attention path (the DRAM counters in
+    profiles/traffic.json are reported only while this digest matches)."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "cached_split_attention_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(csrc, name), "rb").read())
+    return h.hexdigest()
+
+
 def native(args, world, rank, local):
     import torch
     if world > 1:
@@ -398,7 +411,8 @@ def native(args, world, rank, local):
     traffic = None
     try:
         prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-        if prof.get("workload") == args.workload:
+        # counters only count for the kernel source they were taken on
+        if prof.get("workload") == args.workload and prof.get("kernel_source_sha256") == kernel_source_digest():
             traffic = prof.get("dram_bytes_per_recompute_launch")
     except Exception:
         pass
