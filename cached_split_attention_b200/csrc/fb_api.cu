@@ -12,7 +12,7 @@
 #include <string>
 #include <unordered_map>
 
-#include "fb_kernels.cuh"
+#include "fb_tc_kernel.cuh"
 #include "flashblock.h"
 
 namespace {
@@ -81,6 +81,8 @@ fb_status check_ptr(const void* ptr, const char* name, bool needed) {
 
 struct Plan {
   int d = 0, g = 0, wm = 0, tr = 0, tiles = 0, n_groups = 0, splits = 1, threads = 0, smem = 0;
+  bool tc = false;  // tensor-core kernel (tcgen05): head_dim 128, more than 64 rows per group
+  int bn = fb::kBN;  // keys per pipeline chunk (TMA box rows)
   size_t off_grid_ctr = 0, off_cos = 0, bytes = 0;
 };
 
@@ -139,13 +141,22 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only) {
   pl.g = p->num_heads_q / p->num_heads_kv;
   const long rows = static_cast<long>(pl.g) * p->max_q;
   pl.wm = rows <= 16 ? 1 : rows <= 32 ? 2 : rows <= 64 ? 4 : 8;
-  const Shape sh = shape_for(pl.d, pl.wm);
-  pl.threads = sh.threads;
-  pl.smem = sh.smem;
-  pl.tr = 16 * pl.wm;
+  pl.tc = pl.d == 128 && rows > 64;
+  if (pl.tc) {
+    pl.threads = fb::tc::kThreads;
+    pl.smem = fb::tc::kSmem;
+    pl.tr = fb::tc::kM;
+    pl.bn = fb::tc::kN;
+  } else {
+    const Shape sh = shape_for(pl.d, pl.wm);
+    pl.threads = sh.threads;
+    pl.smem = sh.smem;
+    pl.tr = 16 * pl.wm;
+    pl.bn = fb::kBN;
+  }
   pl.tiles = static_cast<int>(std::max<long>(1, (rows + pl.tr - 1) / pl.tr));
   pl.n_groups = p->num_seqs * p->num_heads_kv * pl.tiles;
-  const int chunks = std::max(1, (p->max_kv_out + fb::kBN - 1) / fb::kBN);
+  const int chunks = std::max(1, (p->max_kv_out + pl.bn - 1) / pl.bn);
   int splits = 1;
   if (!in_only) {
     if (p->out_splits > 0) {
@@ -195,13 +206,13 @@ fb_status get_encode(EncodeTiledFn* fn) {
 
 // Map of a THD bf16 buffer [tokens, hkv, d] viewed as 2-D {hkv*d, tokens}; the box
 // is 64 columns (128 bytes, the swizzle span) by kBN token rows.
-fb_status kv_map(const void* ptr, int tokens, int hkv, int d, CUtensorMap* out) {
+fb_status kv_map(const void* ptr, int tokens, int hkv, int d, int box_rows, CUtensorMap* out) {
   std::memset(out, 0, sizeof(*out));
   if (tokens <= 0) return FB_OK;  // never read: every key range is empty
   int dev = 0;
   cudaGetDevice(&dev);
   char key[96];
-  snprintf(key, sizeof(key), "%d:%p:%d:%d:%d", dev, ptr, tokens, hkv, d);
+  snprintf(key, sizeof(key), "%d:%p:%d:%d:%d:%d", dev, ptr, tokens, hkv, d, box_rows);
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -214,7 +225,7 @@ fb_status kv_map(const void* ptr, int tokens, int hkv, int d, CUtensorMap* out) 
   FB_TRY(get_encode(&enc));
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(hkv) * d, static_cast<cuuint64_t>(tokens)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(hkv) * d * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(fb::kBN)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -231,12 +242,12 @@ fb_status kv_map(const void* ptr, int tokens, int hkv, int d, CUtensorMap* out) 
 fb_status launch_attn(const Plan& pl, fb::Params& prm, cudaStream_t stream) {
   const int n_ctas = pl.n_groups * pl.splits;
   if (n_ctas <= 0) return FB_OK;
-  void* fn = shape_for(pl.d, pl.wm).fn;
+  void* fn = pl.tc ? reinterpret_cast<void*>(&fb::tc_attn_kernel) : shape_for(pl.d, pl.wm).fn;
   static std::mutex mu;
-  static bool attr_done[2][9] = {};
+  static bool attr_done[3][9] = {};
   {
     std::lock_guard<std::mutex> lk(mu);
-    bool& done = attr_done[pl.d == 128][pl.wm];
+    bool& done = attr_done[pl.tc ? 2 : (pl.d == 128)][pl.wm];
     if (!done) {
       cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -330,8 +341,8 @@ fb_status fb_out_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16
   std::memset(&prm, 0, sizeof(prm));
   fill_problem(problem, pl, prm);
   fill_workspace(pl, workspace, prm);
-  FB_TRY(kv_map(k_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, &prm.tm_k_out));
-  FB_TRY(kv_map(v_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, &prm.tm_v_out));
+  FB_TRY(kv_map(k_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_k_out));
+  FB_TRY(kv_map(v_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_v_out));
   prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
   prm.do_out = 1;
   prm.head_mask = head_mask;
@@ -354,8 +365,8 @@ fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16*
   fb::Params prm;
   std::memset(&prm, 0, sizeof(prm));
   fill_problem(problem, pl, prm);
-  FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, &prm.tm_k_in));
-  FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, &prm.tm_v_in));
+  FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_k_in));
+  FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_v_in));
   prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
   prm.do_in = 1;
   prm.a_in = a_in;
@@ -435,10 +446,10 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   std::memset(&prm, 0, sizeof(prm));
   fill_problem(problem, pl, prm);
   fill_workspace(pl, workspace, prm);
-  FB_TRY(kv_map(k_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, &prm.tm_k_out));
-  FB_TRY(kv_map(v_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, &prm.tm_v_out));
-  FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, &prm.tm_k_in));
-  FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, &prm.tm_v_in));
+  FB_TRY(kv_map(k_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_k_out));
+  FB_TRY(kv_map(v_out, problem->total_kv_out, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_v_out));
+  FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_k_in));
+  FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_v_in));
 
   if (head_gate && rows) {
     float* cos_ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_cos);

@@ -28,6 +28,16 @@ def _problems():
     # MHA with row tiles of 128 rows (several tiles per group)
     p = W.make_problem([np.arange(150)], [300], [150], 2, 2, 128)
     out.append(("mha_multi_tile", p, 1.0))
+    # tensor-core path: 3 row tiles (128, 128, 44), 8 prefix chunks of 128 keys
+    # (the last one 104 keys), 3 block chunks (the last one 44 keys)
+    p = W.make_problem([np.arange(300)], [1000], [300], 2, 2, 128)
+    out.append(("mha_tc_ragged", p, 1.0))
+    # the same with sharp scores: the running max jumps, O is rescaled in TMEM
+    out.append(("mha_tc_sharp", p, 40.0))
+    # tensor-core path, GQA g=4: 2 sequences, 64 and 37 active rows in permuted
+    # block order (256 and 148 rows), prefixes 777 and 129
+    p = W.make_problem([rng.permutation(64), rng.permutation(80)[:37]], [777, 129], [64, 80], 8, 2, 128)
+    out.append(("gqa4_tc_two_tiles", p, 1.0))
     return out
 
 
