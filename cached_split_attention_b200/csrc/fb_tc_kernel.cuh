@@ -10,24 +10,32 @@
 // log-space merge through distributed shared memory.  What changes is the inner
 // loop, per 128-key chunk:
 //
-//   warp 4 (one thread)  TMA: K chunk -> ring of 2, V chunk -> ring of 2
+//   warp 4 (one thread)  TMA: K chunk -> ring of 3, V chunk -> ring of 3
 //   warp 5 (one thread)  S = Q K^T   (tcgen05.mma, M=128 N=128 K=128, fp32 in TMEM,
 //                                     two S buffers so the next chunk's S overlaps
 //                                     the softmax of this one)
-//                        O += P V    (tcgen05.mma, P from shared memory, O in TMEM;
-//                                     one O accumulator per segment: block, prefix)
+//                        O += P V    (tcgen05.mma with A = P read from TMEM, O in
+//                                     TMEM; one O accumulator per segment)
 //   warps 0-3            one thread per tile row (= TMEM lane): load the S row,
 //                        mask, running max in base 2, P = 2^(s - m) rounded to bf16
-//                        into shared memory; O is rescaled in TMEM only when the
-//                        running max grows by more than 2^8 (the stored max may lag:
-//                        exact, since O and l always share the same reference).
+//                        and stored back over the S row it came from; O is rescaled
+//                        in TMEM only when the running max grows by more than 2^8
+//                        (the stored max may lag: exact, since O and l always share
+//                        the same reference).  Three of every eight 2^x go through a
+//                        cubic on the FMA pipe instead of the MUFU unit, whose
+//                        throughput otherwise bounds the softmax.
+//
+// The MMA thread issues S(c) after P V(c-2) and P V(c) after S(c+1); the tensor
+// core runs them in issue order, so S(c+2) never overwrites P(c) before P V(c) has
+// read it, and the completion of S(c) implies that of P V(c-2).
 //
 // Operand layouts in shared memory are the 128-byte-swizzled tiles TMA writes:
-// Q, K and P are K-major (rows of 64-element halves, 8-row groups 1024 bytes apart),
-// V is MN-major (key rows of 64 d-columns, the two d-halves 16 KB apart).
+// Q and K are K-major (rows of 64-element halves, 8-row groups 1024 bytes apart),
+// V is MN-major (key rows of 64 d-columns, the two d-halves 16 KB apart).  P in
+// TMEM is K-major: lane = row, 32-bit column j = keys 2j (low half), 2j+1.
 //
-// TMEM: 512 columns x 128 lanes: S buffers at columns 0 and 128, prefix O at 256,
-// block O at 384.  Every wait is bounded; on a timeout the CTA records
+// TMEM: 512 columns x 128 lanes: S/P buffers at columns 0 and 128, prefix O at
+// 256, block O at 384.  Every wait is bounded; on a timeout the CTA records
 // kDevTimeout, stops issuing, lets issued copies and MMAs land, and finishes.
 #pragma once
 
@@ -43,12 +51,12 @@ constexpr int kN = 128;           // keys per chunk
 constexpr int kThreads = 192;     // warps 0-3 rows, warp 4 TMA, warp 5 MMA
 constexpr int kHalf = kN * 128;   // 64 columns (128 bytes) x 128 rows: 16 KB
 constexpr int kTile = 2 * kHalf;  // 128 x 128 bf16: 32 KB
+constexpr int kStages = 3;        // K and V rings
 constexpr int kOffK = 0;
-constexpr int kOffV = kOffK + 2 * kTile;
-constexpr int kOffP = kOffV + 2 * kTile;
-constexpr int kOffQ = kOffP + kTile;
+constexpr int kOffV = kOffK + kStages * kTile;
+constexpr int kOffQ = kOffV + kStages * kTile;
 constexpr int kOffBar = kOffQ + kTile;
-constexpr int kNumBars = 16;
+constexpr int kNumBars = 20;
 constexpr int kOffPos = kOffBar + kNumBars * 8;
 constexpr int kOffMisc = kOffPos + kM * 4;
 constexpr int kSmem = 1024 + kOffMisc + 16;  // + alignment of the base to 1024 bytes
@@ -68,11 +76,44 @@ constexpr uint32_t kColIn = 384;
 constexpr uint32_t kIdescS = idesc_bf16(kM, kN, false);
 constexpr uint32_t kIdescO = idesc_bf16(kM, kD, true);
 constexpr float kRescaleSlack = 8.f;  // log2 units the stored running max may lag
+// 2^f on [-1/2, 1/2] by a cubic of least maximum relative error (7.5e-5, far below
+// the bf16 rounding of P); fitted by fit_exp2_poly.py beside this file.
+constexpr float kExpC0 = 0.9999281167984009f;
+constexpr float kExpC1 = 0.6932609677314758f;
+constexpr float kExpC2 = 0.24261054396629333f;
+constexpr float kExpC3 = 0.05517132207751274f;
 
 static_assert(2 * kPartFloats * 4 <= kOffQ, "both partials fit below the Q tile");
 static_assert(kOffPartIn % 16 == 0, "aligned partial");
 static_assert(kM * kWt * 4 <= kTile, "merge table fits in the Q tile");
 static_assert(kSmem <= 232448, "shared memory per CTA");
+
+// 2^x for a pair of x on the FMA pipe: x = j + f with j = round(x) (the
+// 1.5 * 2^23 shifter leaves j in the low mantissa bits of t), 2^f by the cubic,
+// 2^j added to the exponent field.  Inputs below -126 give results below 2^-126
+// (0 for practical purposes).
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& p0, float& p1) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t x = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t shift = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = fadd2(x, shift);
+  const uint64_t f = fsub2(x, fsub2(t, shift));
+  uint64_t q = ffma2(f2_pack(kExpC3, kExpC3), f, f2_pack(kExpC2, kExpC2));
+  q = ffma2(q, f, f2_pack(kExpC1, kExpC1));
+  q = ffma2(q, f, f2_pack(kExpC0, kExpC0));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 }  // namespace tc
 
@@ -81,15 +122,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* k_full = bars;        // [2] TMA -> MMA
-  uint64_t* k_empty = bars + 2;   // [2] MMA -> TMA
-  uint64_t* v_full = bars + 4;    // [2]
-  uint64_t* v_empty = bars + 6;   // [2]
-  uint64_t* s_full = bars + 8;    // [2] MMA -> rows
-  uint64_t* s_free = bars + 10;   // [2] rows -> MMA
-  uint64_t* p_full = bars + 12;   // rows -> MMA
-  uint64_t* pv_done = bars + 13;  // MMA -> rows
-  uint64_t* drain = bars + 14;    // MMA -> MMA (all issued MMAs finished)
+  uint64_t* k_full = bars;        // [3] TMA -> MMA
+  uint64_t* k_empty = bars + 3;   // [3] MMA -> TMA
+  uint64_t* v_full = bars + 6;    // [3]
+  uint64_t* v_empty = bars + 9;   // [3]
+  uint64_t* s_full = bars + 12;   // [2] MMA -> rows
+  uint64_t* p_full = bars + 14;   // rows -> MMA
+  uint64_t* pv_done = bars + 15;  // MMA -> rows
+  uint64_t* drain = bars + 16;    // MMA -> MMA (all issued MMAs finished)
   int* s_pos = reinterpret_cast<int*>(smem + kOffPos);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
@@ -191,7 +231,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
 
     const uint64_t pol = l2_policy_evict_first();
     auto load = [&](int c, bool is_v) {
-      const int st = c & 1;
+      const int st = c % kStages;
       const bool seg_in = c < nA;
       const CUtensorMap* map = is_v ? (seg_in ? &p.tm_v_in : &p.tm_v_out) : (seg_in ? &p.tm_k_in : &p.tm_k_out);
       uint64_t* bar = is_v ? &v_full[st] : &k_full[st];
@@ -203,20 +243,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
     };
     // The TMA thread initialises the barriers and starts the stream at once.
     if (warp == 4 && lane == 0) {
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < kStages; ++i) {
         mbar_init(&k_full[i], 1);
         mbar_init(&k_empty[i], 1);
         mbar_init(&v_full[i], 1);
         mbar_init(&v_empty[i], 1);
-        mbar_init(&s_full[i], 1);
-        mbar_init(&s_free[i], kM);
       }
-      mbar_init(p_full, kM);
+      mbar_init(&s_full[0], 1);
+      mbar_init(&s_full[1], 1);
+      mbar_init(p_full, kM / 32);  // one arrival per row warp
       mbar_init(pv_done, 1);
       mbar_init(drain, 1);
       *s_abort = 0;
       fence_barrier_init();
-      for (int c = 0; c < min(2, n_local); ++c) {
+      for (int c = 0; c < min(kStages, n_local); ++c) {
         load(c, false);
         load(c, true);
       }
@@ -261,18 +301,19 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
       if (warp == 4) {
         // ---------------------------------------------------- TMA producer
         if (lane == 0) {
-          int issued_k = min(2, n_local), issued_v = issued_k;
-          for (int c = 2; c < n_local; ++c) {
+          int issued_k = min(kStages, n_local), issued_v = issued_k;
+          for (int c = kStages; c < n_local; ++c) {
             if (*s_abort) break;
-            const int st = c & 1;
-            if (!mbar_wait(&k_empty[st], ((c >> 1) - 1) & 1)) {
+            const int st = c % kStages;
+            const uint32_t ph = (c / kStages - 1) & 1;  // use of the slot by chunk c - kStages
+            if (!mbar_wait(&k_empty[st], ph)) {
               record_status(kDevTimeout);
               *s_abort = 1;
               break;
             }
             load(c, false);
             issued_k = c + 1;
-            if (!mbar_wait(&v_empty[st], ((c >> 1) - 1) & 1)) {
+            if (!mbar_wait(&v_empty[st], ph)) {
               record_status(kDevTimeout);
               *s_abort = 1;
               break;
@@ -281,47 +322,50 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
             issued_v = c + 1;
           }
           if (*s_abort) {  // copies in flight land before the CTA moves on
-            for (int c = max(0, issued_k - 2); c < issued_k; ++c)
-              if (!mbar_wait(&k_full[c & 1], (c >> 1) & 1)) record_status(kDevTimeout);
-            for (int c = max(0, issued_v - 2); c < issued_v; ++c)
-              if (!mbar_wait(&v_full[c & 1], (c >> 1) & 1)) record_status(kDevTimeout);
+            for (int c = max(0, issued_k - kStages); c < issued_k; ++c)
+              if (!mbar_wait(&k_full[c % kStages], (c / kStages) & 1)) record_status(kDevTimeout);
+            for (int c = max(0, issued_v - kStages); c < issued_v; ++c)
+              if (!mbar_wait(&v_full[c % kStages], (c / kStages) & 1)) record_status(kDevTimeout);
           }
         }
       } else if (warp == 5) {
         // ---------------------------------------------------- MMA issuer
         if (lane == 0) {
           const uint32_t q_a = smem_u32(smem + kOffQ);
-          const uint32_t p_a = smem_u32(smem + kOffP);
+          // Descriptors are built once; a K step or a ring slot only moves the
+          // start address (16-byte units in the low bits), so the issue loop is a
+          // handful of integer adds per MMA.
+          const uint64_t dq = sdesc_sw128(q_a, 16, 1024);
+          const uint64_t dk = sdesc_sw128(smem_u32(smem + kOffK), 16, 1024);
+          const uint64_t dv = sdesc_sw128(smem_u32(smem + kOffV), kHalf, 1024);
           auto issue_s = [&](int c) -> bool {
-            const int st = c & 1;
-            if (!mbar_wait(&k_full[st], (c >> 1) & 1)) return false;
-            if (c >= 2 && !mbar_wait(&s_free[st], ((c >> 1) - 1) & 1)) return false;
+            const int st = c % kStages;
+            if (!mbar_wait(&k_full[st], (c / kStages) & 1)) return false;
             tc_fence_after();
-            const uint32_t k_a = smem_u32(smem + kOffK + st * kTile);
-            const uint32_t d = tmem + kColS + st * kN;
+            const uint64_t dks = dk + static_cast<uint64_t>(st * (kTile >> 4));
+            const uint32_t d = tmem + kColS + (c & 1) * kN;
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-              umma_bf16(d, sdesc_sw128(q_a + off, 16, 1024), sdesc_sw128(k_a + off, 16, 1024), kIdescS, kk > 0);
+              const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+              umma_bf16(d, dq + off, dks + off, kIdescS, kk > 0);
             }
-            umma_commit(&s_full[st]);
+            umma_commit(&s_full[c & 1]);
             umma_commit(&k_empty[st]);
             return true;
           };
           auto issue_pv = [&](int c) -> bool {
-            const int st = c & 1;
+            const int st = c % kStages;
             if (!mbar_wait(p_full, c & 1)) return false;
-            if (!mbar_wait(&v_full[st], (c >> 1) & 1)) return false;
+            if (!mbar_wait(&v_full[st], (c / kStages) & 1)) return false;
             tc_fence_after();
-            const uint32_t v_a = smem_u32(smem + kOffV + st * kTile);
+            const uint64_t dvs = dv + static_cast<uint64_t>(st * (kTile >> 4));
+            const uint32_t pt = tmem + kColS + (c & 1) * kN;  // P(c), packed bf16 pairs
             const bool first = c == 0 || c == nA;
             const uint32_t d = tmem + (c < nA ? kColIn : kColOut);
 #pragma unroll
-            for (int kk = 0; kk < kN / 16; ++kk) {
-              const uint32_t a_off = (kk >> 2) * kHalf + (kk & 3) * 32;
-              umma_bf16(d, sdesc_sw128(p_a + a_off, 16, 1024), sdesc_sw128(v_a + kk * 16 * 128, kHalf, 1024),
-                        kIdescO, (first && kk == 0) ? 0u : 1u);
-            }
+            for (int kk = 0; kk < kN / 16; ++kk)
+              umma_bf16_ts(d, pt + kk * 8, dvs + static_cast<uint64_t>((kk * 16 * 128) >> 4), kIdescO,
+                           (first && kk == 0) ? 0u : 1u);
             umma_commit(pv_done);
             umma_commit(&v_empty[st]);
             return true;
@@ -349,36 +393,30 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
         float m = kNegInf, l = 0.f;
         bool ok = true;
         for (int c = 0; c < n_local; ++c) {
-          if (__any_sync(0xffffffffu, *s_abort != 0)) {
-            ok = false;
-            break;
-          }
           if (c == nA && c > 0) {  // block segment done; the prefix segment starts
             m_in = m;
             l_in = l;
             m = kNegInf;
             l = 0.f;
           }
-          const int st = c & 1;
+          const uint32_t sp = lane_base + kColS + (c & 1) * kN;  // S(c), then P(c)
           const bool seg_in = c < nA;
           const int key0 = seg_in ? c * kN : (pa + c - nA) * kN;
           const int valid = min(kN, (seg_in ? n_in : n_out) - key0);
           const bool first = c == 0 || c == nA;
-          if (!__all_sync(0xffffffffu, mbar_wait(&s_full[st], (c >> 1) & 1))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&s_full[c & 1], (c >> 1) & 1))) {
             ok = false;
             break;
           }
           tc_fence_after();
           uint32_t sv[4][32];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) tmem_ld32(lane_base + kColS + st * kN + 32 * i, sv[i]);
+          for (int i = 0; i < 4; ++i) tmem_ld32(sp + 32 * i, sv[i]);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 4; ++i) reg_fence32(sv[i]);
-          tc_fence_before();
-          mbar_arrive(&s_free[st]);
           // Row max of the raw scores (the scale is positive, so it commutes with
-          // the max), eight independent chains folded at the end.
+          // the max), four independent chains of 3-input maxima.
           if (valid < kN) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -387,17 +425,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
                 if (32 * i + k >= valid) sv[i][k] = __float_as_uint(kNegInf);
             }
           }
-          float mxa[8];
-#pragma unroll
-          for (int a = 0; a < 8; ++a) mxa[a] = kNegInf;
+          float mxa[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) mxa[k & 7] = fmaxf(mxa[k & 7], __uint_as_float(sv[i][k]));
+            for (int k = 0; k < 32; k += 2)
+              mxa[(k >> 1) & 3] = max3(mxa[(k >> 1) & 3], __uint_as_float(sv[i][k]), __uint_as_float(sv[i][k + 1]));
           }
-          const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
-                                 fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]))) *
-                           p.scale_log2;
+          const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])) * p.scale_log2;
           const float m_new = fmaxf(m, mx);
           float alpha = 1.f;
           bool resc = false;
@@ -409,31 +444,52 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
             resc = true;
           }
           const float nm = m == kNegInf ? 0.f : -m;
-          // P = 2^(s * scale - m), rounded to bf16 for the P V product; the row sum
-          // in eight independent chains.
-          uint32_t pk[64];
-          float rsa[8];
+          // P = 2^(s * scale - m), rounded to bf16 for the P V product; paired fp32
+          // arithmetic, pairs 8a+0..2 of every eight by the cubic, the rest by MUFU;
+          // the row sum in eight chains (four paired accumulators).
+          uint32_t pk[2][32];  // packed bf16 pairs: keys 2j, 2j+1 in column j
+          uint64_t rsa[4];
 #pragma unroll
-          for (int a = 0; a < 8; ++a) rsa[a] = 0.f;
+          for (int a = 0; a < 4; ++a) rsa[a] = 0ull;
+          const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+          const uint64_t nm2 = f2_pack(nm, nm);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
 #pragma unroll
             for (int k = 0; k < 32; k += 2) {
-              const float p0 = ex2(fmaf(__uint_as_float(sv[i][k]), p.scale_log2, nm));
-              const float p1 = ex2(fmaf(__uint_as_float(sv[i][k + 1]), p.scale_log2, nm));
-              rsa[(k >> 1) & 7] += p0 + p1;
-              pk[16 * i + k / 2] = pack_bf16x2(p0, p1);
+              const uint64_t x = ffma2(f2_pack(__uint_as_float(sv[i][k]), __uint_as_float(sv[i][k + 1])), scale2, nm2);
+              float p0, p1;
+              if (((k >> 1) & 7) < 3) {
+                exp2_poly2(x, p0, p1);
+              } else {
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              rsa[(k >> 1) & 3] = fadd2(rsa[(k >> 1) & 3], f2_pack(p0, p1));
+              pk[i >> 1][(16 * i + k / 2) & 31] = pack_bf16x2(p0, p1);
             }
           }
-          const float rs = ((rsa[0] + rsa[1]) + (rsa[2] + rsa[3])) + ((rsa[4] + rsa[5]) + (rsa[6] + rsa[7]));
+          float r0, r1, r2, r3, r4, r5, r6, r7;
+          f2_unpack(rsa[0], r0, r1);
+          f2_unpack(rsa[1], r2, r3);
+          f2_unpack(rsa[2], r4, r5);
+          f2_unpack(rsa[3], r6, r7);
+          const float rs = ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
           l = l * alpha + rs;
-          // the previous chunk's P V has finished: O may be rescaled, P rewritten
-          if (c > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (c - 1) & 1))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, resc)) {
+          // P V(c-1) must be finished before O is rescaled; otherwise the wait only
+          // keeps the rows in step with the MMA thread (one wait per chunk, before
+          // P(c) is published, so the phase waited for is never overtaken).
+          const bool rescale = __any_sync(0xffffffffu, resc);
+          bool waited = c == 0;
+          if (rescale) {
+            if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (c - 1) & 1))) {
+              ok = false;
+              break;
+            }
+            waited = true;
+            tc_fence_after();
             const uint32_t oc = lane_base + (seg_in ? kColIn : kColOut);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -445,22 +501,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
               for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
               tmem_st32(oc + 32 * i, o);
             }
-            tmem_wait_st();
           }
-          // P row -> shared memory (K-major, 128-byte swizzle, two 64-key halves)
-          uint8_t* prow = smem + kOffP + r * 128;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              const int w0 = 32 * h + 4 * cc;
-              *reinterpret_cast<uint4*>(prow + h * kHalf + ((cc ^ (r & 7)) << 4)) =
-                  make_uint4(pk[w0], pk[w0 + 1], pk[w0 + 2], pk[w0 + 3]);
+          // P(c) over the S(c) columns it came from (read above, by this thread)
+          tmem_st32(sp, pk[0]);
+          tmem_st32(sp + 32, pk[1]);
+          tmem_wait_st();
+          if (!waited) {
+            if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (c - 1) & 1))) {
+              ok = false;
+              break;
             }
           }
-          fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(p_full);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full);
         }
         if (ok && !__all_sync(0xffffffffu, mbar_wait(pv_done, (n_local - 1) & 1))) ok = false;
         if (!ok) {
