@@ -12,7 +12,7 @@
 #include <string>
 #include <unordered_map>
 
-#include "fb_tc_kernel.cuh"
+#include "fb_tc2_kernel.cuh"
 #include "flashblock.h"
 
 namespace {
@@ -81,7 +81,8 @@ fb_status check_ptr(const void* ptr, const char* name, bool needed) {
 
 struct Plan {
   int d = 0, g = 0, wm = 0, tr = 0, tiles = 0, n_groups = 0, splits = 1, threads = 0, smem = 0;
-  bool tc = false;  // tensor-core kernel (tcgen05): head_dim 128, more than 64 rows per group
+  bool tc = false;   // tensor-core kernel (tcgen05): head_dim 128, more than 64 rows per group
+  bool tc2 = false;  // two-tile tensor-core kernel: fused step, MHA, at least 256 rows per head
   int bn = fb::kBN;  // keys per pipeline chunk (TMA box rows)
   size_t off_grid_ctr = 0, off_cos = 0, bytes = 0;
 };
@@ -135,14 +136,23 @@ Shape shape_for(int d, int wm) {
 }
 
 // in_only: fb_in_attn (no prefix pass, one CTA per group)
-Plan make_plan(const fb_problem* p, int num_sms, bool in_only) {
+// Groups of at least this many rows (head_dim 128) go to the tensor-core kernel.
+int kTcMinRows = 65;
+
+Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = false) {
   Plan pl;
   pl.d = p->head_dim;
   pl.g = p->num_heads_q / p->num_heads_kv;
   const long rows = static_cast<long>(pl.g) * p->max_q;
   pl.wm = rows <= 16 ? 1 : rows <= 32 ? 2 : rows <= 64 ? 4 : 8;
-  pl.tc = pl.d == 128 && rows > 64;
-  if (pl.tc) {
+  pl.tc = pl.d == 128 && rows >= kTcMinRows;
+  pl.tc2 = fused && pl.d == 128 && pl.g == 1 && p->max_q >= 2 * fb::tc2::kM;
+  if (pl.tc2) {
+    pl.threads = fb::tc2::kThreads;
+    pl.smem = fb::tc2::kSmem;
+    pl.tr = 2 * fb::tc2::kM;
+    pl.bn = fb::tc2::kN;
+  } else if (pl.tc) {
     pl.threads = fb::tc::kThreads;
     pl.smem = fb::tc::kSmem;
     pl.tr = fb::tc::kM;
@@ -158,7 +168,7 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only) {
   pl.n_groups = p->num_seqs * p->num_heads_kv * pl.tiles;
   const int chunks = std::max(1, (p->max_kv_out + pl.bn - 1) / pl.bn);
   int splits = 1;
-  if (!in_only) {
+  if (!in_only && !pl.tc2) {
     if (p->out_splits > 0) {
       splits = p->out_splits;
     } else {
@@ -242,12 +252,14 @@ fb_status kv_map(const void* ptr, int tokens, int hkv, int d, int box_rows, CUte
 fb_status launch_attn(const Plan& pl, fb::Params& prm, cudaStream_t stream) {
   const int n_ctas = pl.n_groups * pl.splits;
   if (n_ctas <= 0) return FB_OK;
-  void* fn = pl.tc ? reinterpret_cast<void*>(&fb::tc_attn_kernel) : shape_for(pl.d, pl.wm).fn;
+  void* fn = pl.tc2  ? reinterpret_cast<void*>(&fb::tc2_attn_kernel)
+             : pl.tc ? reinterpret_cast<void*>(&fb::tc_attn_kernel)
+                     : shape_for(pl.d, pl.wm).fn;
   static std::mutex mu;
-  static bool attr_done[3][9] = {};
+  static bool attr_done[4][9] = {};
   {
     std::lock_guard<std::mutex> lk(mu);
-    bool& done = attr_done[pl.tc ? 2 : (pl.d == 128)][pl.wm];
+    bool& done = attr_done[pl.tc2 ? 3 : pl.tc ? 2 : (pl.d == 128)][pl.wm];
     if (!done) {
       cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -437,7 +449,7 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   if (problem->num_seqs > 0 && !cache->valid) return fail(FB_ERR_INVALID_ARG, "cache->valid is NULL");
   if (cache->q_ref) FB_TRY(check_ptr(cache->q_ref, "cache->q_ref", true));
   if (problem->num_seqs == 0) return FB_OK;
-  const Plan pl = make_plan(problem, device_sms(), false);
+  const Plan pl = make_plan(problem, device_sms(), false, true);
   if (!workspace || workspace_bytes < pl.bytes)
     return fail(FB_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, pl.bytes);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

