@@ -137,7 +137,7 @@ Shape shape_for(int d, int wm) {
 
 // in_only: fb_in_attn (no prefix pass, one CTA per group)
 // Groups of at least this many rows (head_dim 128) go to the tensor-core kernel.
-int kTcMinRows = 65;
+constexpr int kTcMinRows = 65;
 
 Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = false) {
   Plan pl;
@@ -272,19 +272,40 @@ fb_status launch_attn(const Plan& pl, fb::Params& prm, cudaStream_t stream) {
   cfg.blockDim = dim3(pl.threads);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (pl.splits > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = pl.splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = pl.splits;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
   void* args[] = {&prm};
   cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
   return FB_OK;
+}
+
+// Launch of a kernel without clusters, allowed to start while the previous
+// kernel of the stream finishes (each kernel waits for it before reading).
+template <typename Arg>
+cudaError_t launch_pdl(void (*fn)(Arg), int blocks, int threads, cudaStream_t stream, const Arg& arg) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(threads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  Arg a = arg;
+  void* args[] = {&a};
+  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(fn), args);
 }
 
 void fill_problem(const fb_problem* p, const Plan& pl, fb::Params& prm) {
@@ -396,8 +417,7 @@ fb_status fb_merge(int64_t n, int32_t d, const float* a_out, const float* l_out,
                      l_full};
   const int64_t total = n * static_cast<int64_t>(d);
   const int blocks = static_cast<int>(std::min<int64_t>((total + 255) / 256, 148 * 16));
-  fb::merge_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(mp);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(fb::merge_kernel, blocks, 256, reinterpret_cast<cudaStream_t>(stream), mp);
   if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
   return FB_OK;
 }
@@ -413,9 +433,8 @@ fb_status fb_head_similarity(const fb_problem* problem, const fb_bf16* q, const 
                    problem->cu_seqlens_q, problem->q_rows,
                    problem->cu_seqlens_kv_in, reinterpret_cast<const __nv_bfloat16*>(q),
                    reinterpret_cast<const __nv_bfloat16*>(q_ref), cos_out};
-  fb::similarity_kernel<<<problem->num_seqs * problem->num_heads_q, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      sp);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(fb::similarity_kernel, problem->num_seqs * problem->num_heads_q, 256,
+                             reinterpret_cast<cudaStream_t>(stream), sp);
   if (e != cudaSuccess) return cuda_fail(e, "similarity kernel launch");
   return FB_OK;
 }

@@ -27,6 +27,17 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
+// ------------------------------------------------------------------ dependent launch
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream is finishing;
+// pdl_wait() returns once that kernel has completed and its writes are visible
+// (at once when there is no such kernel), so every kernel here calls it before
+// its first global read.  pdl_trigger() lets the next such kernel launch: its
+// CTAs take free SMs and wait in their own pdl_wait().
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

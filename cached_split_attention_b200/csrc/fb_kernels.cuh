@@ -340,6 +340,8 @@ __device__ __forceinline__ void consume_keys(Acc<D>& acc, const uint32_t (&qf)[D
 
 template <int D, int WM, int WN, int STAGES>
 __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kernel(const __grid_constant__ Params p) {
+  pdl_wait();
+  pdl_trigger();
   using C = Cfg<D, WM, WN, STAGES>;
   constexpr int TR = C::kRows;
   constexpr int KW = C::kKW;
@@ -829,6 +831,8 @@ struct SimParams {
 // cos(Q_bh, q_ref_bh) over the active rows x d of (b, h); one CTA per (b, h).
 // Fixed order: each thread accumulates a fixed strided subset, then a fixed tree.
 __global__ void __launch_bounds__(256) similarity_kernel(const SimParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x / p.hq;
   const int h = blockIdx.x % p.hq;
   const int q0 = p.cu_q[b];
@@ -906,6 +910,8 @@ struct MergeParams {
 };
 
 __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t total = p.n * p.d;
   for (int64_t idx = blockIdx.x * 256ll + threadIdx.x; idx < total; idx += static_cast<int64_t>(gridDim.x) * 256) {
     const int64_t e = idx / p.d;

@@ -61,6 +61,8 @@ static_assert(kSmem <= 232448, "shared memory per CTA");
 }  // namespace tc2
 
 __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid_constant__ Params p) {
+  pdl_wait();
+  pdl_trigger();
   using namespace tc2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

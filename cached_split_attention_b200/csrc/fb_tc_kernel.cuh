@@ -118,6 +118,8 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }  // namespace tc
 
 __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_constant__ Params p) {
+  pdl_wait();
+  pdl_trigger();
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
