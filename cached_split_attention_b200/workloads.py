@@ -30,6 +30,7 @@ GATE_TAU = 1
 GATE_HEAD = 2
 FORCE_RECOMPUTE = 4
 FORCE_REUSE = 8
+GATE_TAU_CUM = 16  # tau gate on the updated tokens summed since the last recompute
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -15,6 +15,12 @@ cached out-of-block partial (A_out, L_out) is reused or recomputed:
     query and gets no output, but its K/V stay in the block and are still attended.
     The active set only shrinks.
 
+Cumulative variant of the threshold gate (a reading of "the number of updated
+tokens"; the pages count them per step): with GATE_TAU_CUM, M is the number of
+block tokens updated since the head's cache was built, i.e. the per-step counts
+summed over the steps since the head's last recompute, this step included; a
+recompute starts the count again from zero.
+
 Readings taken where the pages are silent: gates combine with AND on "reuse"; a
 cache that was never filled (or was invalidated) always recomputes, overriding a
 forced reuse; FORCE_RECOMPUTE overrides everything; a caller-supplied per-head
@@ -36,6 +42,7 @@ GATE_TAU = 1
 GATE_HEAD = 2
 FORCE_RECOMPUTE = 4
 FORCE_REUSE = 8
+GATE_TAU_CUM = 16
 
 
 @dataclasses.dataclass
@@ -43,18 +50,21 @@ class OracleCache:
     """(A_out, L_out) per block position and q-head, plus bookkeeping.
 
     a_out [total_kv_in, H_q, d], l_out [total_kv_in, H_q], valid [num_seqs, H_q],
-    q_ref [total_kv_in, H_q, d]: the queries each head's cache was built with."""
+    q_ref [total_kv_in, H_q, d]: the queries each head's cache was built with,
+    m_acc [num_seqs, H_q]: block tokens updated since the head's last recompute
+    (GATE_TAU_CUM)."""
     a_out: np.ndarray
     l_out: np.ndarray
     valid: np.ndarray
     q_ref: np.ndarray
+    m_acc: np.ndarray = None
 
     @classmethod
     def empty(cls, problem):
         T, H, d = problem.total_kv_in, problem.num_heads_q, problem.head_dim
         return cls(a_out=np.full((T, H, d), np.nan), l_out=np.full((T, H), np.nan),
                    valid=np.zeros((problem.num_seqs, H), dtype=bool),
-                   q_ref=np.zeros((T, H, d)))
+                   q_ref=np.zeros((T, H, d)), m_acc=np.zeros((problem.num_seqs, H), dtype=np.int64))
 
 
 def cache_rows(problem) -> np.ndarray:
@@ -83,8 +93,10 @@ def head_cosine(problem, q: np.ndarray, q_ref: np.ndarray) -> np.ndarray:
 
 
 def decide(flags: int, tau: int, gamma: float, valid: np.ndarray, n_updated: np.ndarray,
-           cos: Optional[np.ndarray] = None, head_reuse_in: Optional[np.ndarray] = None) -> np.ndarray:
-    """recompute[b, h] (bool) from the gate inputs; see the module docstring."""
+           cos: Optional[np.ndarray] = None, head_reuse_in: Optional[np.ndarray] = None,
+           m_acc: Optional[np.ndarray] = None) -> np.ndarray:
+    """recompute[b, h] (bool) from the gate inputs; see the module docstring.
+    ``m_acc`` [num_seqs, H_q] is the cumulative count before this step (GATE_TAU_CUM)."""
     valid = np.asarray(valid, dtype=bool)
     S, H = valid.shape
     if flags & FORCE_RECOMPUTE:
@@ -98,9 +110,21 @@ def decide(flags: int, tau: int, gamma: float, valid: np.ndarray, n_updated: np.
         if flags & GATE_TAU:
             m = np.asarray(n_updated, dtype=np.int64)
             reuse &= (m < int(tau))[:, None]
+        if flags & GATE_TAU_CUM:
+            m = np.asarray(m_acc, dtype=np.int64) + np.asarray(n_updated, dtype=np.int64)[:, None]
+            reuse &= m < int(tau)
         if flags & GATE_HEAD:
             reuse &= np.asarray(cos) > np.float64(gamma)
     return ~(reuse & valid)
+
+
+def next_m_acc(flags: int, m_acc: np.ndarray, n_updated: np.ndarray, recompute: np.ndarray) -> np.ndarray:
+    """Cumulative count after a step: 0 where the head recomputed, else the old
+    count plus this step's updates (kept whenever GATE_TAU_CUM is set)."""
+    if not flags & GATE_TAU_CUM:
+        return np.asarray(m_acc)
+    grown = np.asarray(m_acc, dtype=np.int64) + np.asarray(n_updated, dtype=np.int64)[:, None]
+    return np.where(recompute, 0, grown)
 
 
 @dataclasses.dataclass
@@ -149,7 +173,10 @@ def run_policy(workload, sample: Optional[Sequence[Tuple[int, int]]] = None,
         if flags & GATE_HEAD:
             cos = head_cosine(p, q, cache.q_ref)
         hr = None if head_reuse_in is None else head_reuse_in[s]
-        rec = decide(flags, workload.tau, workload.gamma, cache.valid, st.n_updated, cos, hr)
+        if cache.m_acc is None:
+            cache.m_acc = np.zeros(cache.valid.shape, dtype=np.int64)
+        rec = decide(flags, workload.tau, workload.gamma, cache.valid, st.n_updated, cos, hr, cache.m_acc)
+        cache.m_acc = next_m_acc(flags, cache.m_acc, st.n_updated, rec)
         rows = _sample_rows(p, sample)
         crow = cache_rows(p)
         # recompute the out-of-block partial where the gates say so

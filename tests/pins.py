@@ -188,6 +188,33 @@ def check_golden_gates(decide):
     assert rec.all(), "tau failure must recompute regardless of cos"
 
 
+def check_cumulative_gate(decide, next_m_acc):
+    """The GATE_TAU_CUM sequence of tests/golden/gates.txt, step by step; plus the
+    per-sequence broadcast of n_updated over heads and the reset on any recompute."""
+    g = load("gates.txt")
+    tau = int(g["cum_tau"][0])
+    steps = g["cum_steps"].reshape(-1, 3)
+    valid = np.zeros((1, 1), bool)
+    m_acc = np.zeros((1, 1), np.int64)
+    for s, (n, exp_rec, exp_m) in enumerate(steps):
+        rec = decide(16, tau, 0.0, valid, np.array([int(n)]), None, None, m_acc)
+        assert bool(rec[0, 0]) == bool(exp_rec), ("cumulative step", s, rec, exp_rec)
+        m_acc = next_m_acc(16, m_acc, np.array([int(n)]), rec)
+        assert int(m_acc[0, 0]) == int(exp_m), ("cumulative count", s, m_acc, exp_m)
+        valid = valid | rec
+    # two sequences x two heads: counts differ per head, updates per sequence
+    m_acc = np.array([[0, 3], [2, 1]])
+    rec = decide(16, 4, 0.0, np.ones((2, 2), bool), np.array([1, 2]), None, None, m_acc)
+    assert rec.tolist() == [[False, True], [True, False]], rec
+    nxt = next_m_acc(16, m_acc, np.array([1, 2]), rec)
+    assert nxt.tolist() == [[1, 0], [0, 3]], nxt
+    # a forced recompute resets the count; a caller mask replaces the gate
+    rec = decide(16 | 4, 4, 0.0, np.ones((1, 1), bool), np.array([0]), None, None, np.array([[1]]))
+    assert rec.all() and next_m_acc(16, np.array([[1]]), np.array([0]), rec).tolist() == [[0]]
+    # without the flag the count is not kept
+    assert next_m_acc(1, np.array([[5]]), np.array([3]), np.array([[False]])).tolist() == [[5]]
+
+
 def check_cosine(head_cosine):
     """cos(x, x) = 1, cos(x, -x) = -1, cos(x, 2x) = 1, orthogonal rows = 0, over the
     active rows of each sequence only (cache rows addressed by block position)."""

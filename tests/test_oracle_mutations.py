@@ -64,6 +64,19 @@ DECIDE_MUTANTS = [
     ("force reuse ignored", "if flags & FORCE_REUSE:", "if flags & 0:"),
 ]
 
+CUMULATIVE_MUTANTS = [
+    ("cumulative: <= instead of <", "reuse &= m < int(tau)", "reuse &= m <= int(tau)"),
+    ("cumulative: this step's updates left out", "m = np.asarray(m_acc, dtype=np.int64) + np.asarray(n_updated, dtype=np.int64)[:, None]",
+     "m = np.asarray(m_acc, dtype=np.int64) + 0 * np.asarray(n_updated, dtype=np.int64)[:, None]"),
+]
+
+NEXT_M_MUTANTS = [
+    ("count not reset on recompute", "return np.where(recompute, 0, grown)", "return grown"),
+    ("count reset on reuse", "return np.where(recompute, 0, grown)", "return np.where(recompute, grown, 0)"),
+    ("updates dropped from the count", "grown = np.asarray(m_acc, dtype=np.int64) + np.asarray(n_updated, dtype=np.int64)[:, None]",
+     "grown = np.asarray(m_acc, dtype=np.int64)"),
+]
+
 COSINE_MUTANTS = [
     ("no square root", "den = np.sqrt(np.dot(x, x) * np.dot(y, y))", "den = np.dot(x, x) * np.dot(y, y)"),
     ("cache addressed by packed row", "y = q_ref[crow[r0:r1], h].reshape(-1)", "y = q_ref[r0:r1, h].reshape(-1)"),
@@ -96,6 +109,18 @@ def test_merge_mutants_caught(label, old, new):
 def test_decide_mutants_caught(label, old, new):
     bad = mutate(policy, "decide", old, new)
     assert caught(pins.check_golden_gates, bad), label
+
+
+@pytest.mark.parametrize("label,old,new", CUMULATIVE_MUTANTS, ids=[m[0] for m in CUMULATIVE_MUTANTS])
+def test_cumulative_mutants_caught(label, old, new):
+    bad = mutate(policy, "decide", old, new)
+    assert caught(pins.check_cumulative_gate, bad, policy.next_m_acc), label
+
+
+@pytest.mark.parametrize("label,old,new", NEXT_M_MUTANTS, ids=[m[0] for m in NEXT_M_MUTANTS])
+def test_next_m_mutants_caught(label, old, new):
+    bad = mutate(policy, "next_m_acc", old, new)
+    assert caught(pins.check_cumulative_gate, policy.decide, bad), label
 
 
 @pytest.mark.parametrize("label,old,new", COSINE_MUTANTS, ids=[m[0] for m in COSINE_MUTANTS])

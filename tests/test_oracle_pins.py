@@ -40,3 +40,7 @@ def test_cosine():
 
 def test_problem_level_vs_brute_force():
     pins.check_problem_vs_brute(attention.attend_problem, attention.merge, attention.attend_full)
+
+
+def test_cumulative_gate():
+    pins.check_cumulative_gate(policy.decide, policy.next_m_acc)
