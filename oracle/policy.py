@@ -127,6 +127,36 @@ def next_m_acc(flags: int, m_acc: np.ndarray, n_updated: np.ndarray, recompute: 
     return np.where(recompute, 0, grown)
 
 
+def cache_invalidate_seqs(cache: OracleCache, seq_mask) -> None:
+    """Refresh of some branches (BlockBatch, "Methodologie : BlockBatch", item 3:
+    periodic full-sequence refreshes recompute the K/V of the branches): the
+    FlashBlock entries of the marked sequences become empty and their cumulative
+    counts restart."""
+    m = np.asarray(seq_mask, dtype=bool)
+    cache.valid[m] = False
+    if cache.m_acc is not None:
+        cache.m_acc[m] = 0
+
+
+def cache_copy_seq(cache: OracleCache, problem, src: int, dst: int) -> None:
+    """Leader-based synchronisation (BlockBatch, "Methodologie : BlockBatch", item 2:
+    a lagging branch copies the leader's sequence state and K/V cache): the entries
+    of block positions 0..min(B_src, B_dst)-1 of every head are copied from sequence
+    src to sequence dst, with the validity and count of each head.  When dst has
+    more block positions than src, those it cannot fill leave its heads empty."""
+    if src == dst:
+        return
+    s0, s1 = int(problem.cu_seqlens_kv_in[src]), int(problem.cu_seqlens_kv_in[src + 1])
+    d0, d1 = int(problem.cu_seqlens_kv_in[dst]), int(problem.cu_seqlens_kv_in[dst + 1])
+    n = min(s1 - s0, d1 - d0)
+    cache.a_out[d0:d0 + n] = cache.a_out[s0:s0 + n]
+    cache.l_out[d0:d0 + n] = cache.l_out[s0:s0 + n]
+    cache.q_ref[d0:d0 + n] = cache.q_ref[s0:s0 + n]
+    cache.valid[dst] = cache.valid[src] & (d1 - d0 <= s1 - s0)
+    if cache.m_acc is not None:
+        cache.m_acc[dst] = cache.m_acc[src]
+
+
 @dataclasses.dataclass
 class StepResult:
     recompute: np.ndarray          # [num_seqs, H_q] bool
