@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libflashblock.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
-GATE_TAU, GATE_HEAD, FORCE_RECOMPUTE, FORCE_REUSE = 1, 2, 4, 8
+GATE_TAU, GATE_HEAD, FORCE_RECOMPUTE, FORCE_REUSE, GATE_TAU_CUM = 1, 2, 4, 8, 16
 
 
 class FlashBlockError(RuntimeError):
@@ -44,7 +44,7 @@ class FbProblem(ctypes.Structure):
 
 class FbCache(ctypes.Structure):
     _fields_ = [("a_out", ctypes.c_void_p), ("l_out", ctypes.c_void_p),
-                ("valid", ctypes.c_void_p), ("q_ref", ctypes.c_void_p)]
+                ("valid", ctypes.c_void_p), ("q_ref", ctypes.c_void_p), ("m_acc", ctypes.c_void_p)]
 
 
 class FbParams(ctypes.Structure):
@@ -69,6 +69,8 @@ def _load():
         "fb_step": (st, [P, ctypes.POINTER(FbParams), ctypes.POINTER(FbCache), vp, vp, vp, vp, vp, vp, vp,
                          vp, vp, vp, vp, sz, vp]),
         "fb_cache_invalidate": (st, [P, ctypes.POINTER(FbCache), vp]),
+        "fb_cache_copy_seq": (st, [P, ctypes.POINTER(FbCache), ctypes.c_int32, ctypes.c_int32, vp]),
+        "fb_cache_invalidate_seqs": (st, [P, ctypes.POINTER(FbCache), vp, vp]),
         "fb_release_cache": (st, []),
         "fb_device_status": (st, [ctypes.POINTER(ctypes.c_int32), vp]),
         "fb_step_noalloc": (st, [P, ctypes.POINTER(FbParams), ctypes.POINTER(FbCache), vp, vp, vp, vp, vp, vp, vp,
@@ -148,7 +150,9 @@ class Cache:
         self.l_out = torch.zeros((max(T, 1), H), dtype=torch.float32, device=device)
         self.valid = torch.zeros((max(problem.num_seqs, 1), H), dtype=torch.uint8, device=device)
         self.q_ref = torch.zeros((max(T, 1), H, d), dtype=torch.bfloat16, device=device) if with_q_ref else None
-        self.struct = FbCache(_ptr(self.a_out), _ptr(self.l_out), _ptr(self.valid), _ptr(self.q_ref))
+        self.m_acc = torch.zeros((max(problem.num_seqs, 1), H), dtype=torch.int32, device=device)
+        self.struct = FbCache(_ptr(self.a_out), _ptr(self.l_out), _ptr(self.valid), _ptr(self.q_ref),
+                              _ptr(self.m_acc))
 
     @property
     def ref(self):
@@ -219,6 +223,14 @@ def step_noalloc(problem: DeviceProblem, prm: FbParams, cache: Cache, q, k_in, v
 
 def cache_invalidate(problem: DeviceProblem, cache: Cache, stream=None):
     _check(_lib.fb_cache_invalidate(problem.ref, cache.ref, _stream(stream)))
+
+
+def cache_copy_seq(problem: DeviceProblem, cache: Cache, src_seq: int, dst_seq: int, stream=None):
+    _check(_lib.fb_cache_copy_seq(problem.ref, cache.ref, int(src_seq), int(dst_seq), _stream(stream)))
+
+
+def cache_invalidate_seqs(problem: DeviceProblem, cache: Cache, seq_mask=None, stream=None):
+    _check(_lib.fb_cache_invalidate_seqs(problem.ref, cache.ref, _ptr(seq_mask), _stream(stream)))
 
 
 def release_cache():

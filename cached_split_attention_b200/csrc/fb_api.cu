@@ -447,9 +447,13 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   if (!params) return fail(FB_ERR_INVALID_ARG, "params is NULL");
   if (!cache) return fail(FB_ERR_INVALID_ARG, "cache is NULL");
   const unsigned flags = params->flags;
-  if (flags & ~15u) return fail(FB_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags & ~15u);
+  if (flags & ~31u) return fail(FB_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags & ~31u);
   if ((flags & FB_FORCE_RECOMPUTE) && (flags & FB_FORCE_REUSE))
     return fail(FB_ERR_INVALID_ARG, "FB_FORCE_RECOMPUTE and FB_FORCE_REUSE are exclusive");
+  if ((flags & FB_GATE_TAU) && (flags & FB_GATE_TAU_CUM))
+    return fail(FB_ERR_INVALID_ARG, "FB_GATE_TAU and FB_GATE_TAU_CUM are exclusive");
+  if ((flags & FB_GATE_TAU_CUM) && problem->num_seqs > 0 && (!n_updated || !cache->m_acc))
+    return fail(FB_ERR_INVALID_ARG, "FB_GATE_TAU_CUM needs n_updated and cache->m_acc");
   const bool rows = problem->total_q > 0;
   const bool uses_gates = !(flags & (FB_FORCE_RECOMPUTE | FB_FORCE_REUSE)) && !head_reuse_in;
   const bool head_gate = uses_gates && (flags & FB_GATE_HEAD);
@@ -499,6 +503,7 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   prm.cache_a = cache->a_out;
   prm.cache_l = cache->l_out;
   prm.valid = cache->valid;
+  prm.m_acc = cache->m_acc;
   prm.q_ref = reinterpret_cast<__nv_bfloat16*>(cache->q_ref);
   prm.a_full = reinterpret_cast<__nv_bfloat16*>(a_full);
   prm.l_full = l_full;
@@ -513,6 +518,41 @@ fb_status fb_cache_invalidate(const fb_problem* problem, const fb_cache* cache, 
   if (!n) return FB_OK;
   cudaError_t e = cudaMemsetAsync(cache->valid, 0, n, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(valid)");
+  return FB_OK;
+}
+
+fb_status fb_cache_copy_seq(const fb_problem* problem, const fb_cache* cache, int32_t src_seq, int32_t dst_seq,
+                            fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  if (!cache) return fail(FB_ERR_INVALID_ARG, "cache is NULL");
+  if (src_seq < 0 || src_seq >= problem->num_seqs || dst_seq < 0 || dst_seq >= problem->num_seqs)
+    return fail(FB_ERR_INVALID_ARG, "sequence index out of range (src %d, dst %d, num_seqs %d)", src_seq, dst_seq,
+                problem->num_seqs);
+  if (src_seq == dst_seq) return FB_OK;
+  if (!cache->valid) return fail(FB_ERR_INVALID_ARG, "cache->valid is NULL");
+  FB_TRY(check_ptr(cache->a_out, "cache->a_out", problem->total_kv_in > 0));
+  if (problem->total_kv_in > 0 && !cache->l_out) return fail(FB_ERR_INVALID_ARG, "cache->l_out is NULL");
+  if (cache->q_ref) FB_TRY(check_ptr(cache->q_ref, "cache->q_ref", true));
+  fb::CacheCopyParams cp{problem->num_heads_q, problem->head_dim, problem->num_seqs, problem->total_kv_in, src_seq,
+                         dst_seq, problem->cu_seqlens_kv_in, cache->a_out, cache->l_out, cache->valid,
+                         reinterpret_cast<__nv_bfloat16*>(cache->q_ref), cache->m_acc};
+  const long items = static_cast<long>(std::max(problem->max_kv_in, 1)) * problem->num_heads_q * (problem->head_dim / 4);
+  const int blocks = static_cast<int>(std::min<long>((items + 255) / 256, 148 * 8));
+  cudaError_t e = launch_pdl(fb::cache_copy_kernel, std::max(blocks, 1), 256, reinterpret_cast<cudaStream_t>(stream), cp);
+  if (e != cudaSuccess) return cuda_fail(e, "cache copy kernel launch");
+  return FB_OK;
+}
+
+fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* cache, const uint8_t* seq_mask,
+                                   fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  if (!cache || (!cache->valid && problem->num_seqs > 0)) return fail(FB_ERR_INVALID_ARG, "cache->valid is NULL");
+  if (problem->num_seqs == 0) return FB_OK;
+  fb::InvalidateParams ip{problem->num_heads_q, problem->num_seqs, seq_mask, cache->valid, cache->m_acc};
+  const int total = problem->num_seqs * problem->num_heads_q;
+  const int blocks = std::min((total + 255) / 256, 148);
+  cudaError_t e = launch_pdl(fb::cache_invalidate_kernel, blocks, 256, reinterpret_cast<cudaStream_t>(stream), ip);
+  if (e != cudaSuccess) return cuda_fail(e, "cache invalidate kernel launch");
   return FB_OK;
 }
 

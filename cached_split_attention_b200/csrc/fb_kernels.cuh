@@ -38,7 +38,7 @@
 
 namespace fb {
 
-constexpr unsigned kGateTau = 1u, kGateHead = 2u, kForceRecompute = 4u, kForceReuse = 8u;
+constexpr unsigned kGateTau = 1u, kGateHead = 2u, kForceRecompute = 4u, kForceReuse = 8u, kGateTauCum = 16u;
 constexpr int kBN = 64;        // keys per pipeline stage
 constexpr int kMaxGroup = 32;  // q-heads per kv-head
 constexpr int kMaxSplits = 8;  // CTAs per cluster (portable limit)
@@ -77,6 +77,7 @@ struct alignas(64) Params {
   float* cache_a;
   float* cache_l;
   uint8_t* valid;
+  int* m_acc;  // cumulative updated-token count per (b, h) (kGateTauCum)
   __nv_bfloat16* q_ref;
   __nv_bfloat16* a_full;
   float* l_full;
@@ -97,8 +98,47 @@ __device__ __forceinline__ bool head_recompute(const Params& p, int b, int h) {
   if (p.head_reuse_in) return p.head_reuse_in[idx] == 0;
   bool reuse = true;
   if (p.flags & kGateTau) reuse = reuse && (p.n_updated[b] < p.tau);
+  if (p.flags & kGateTauCum) reuse = reuse && (p.m_acc[idx] + p.n_updated[b] < p.tau);
   if (p.flags & kGateHead) reuse = reuse && (p.cos[idx] > p.gamma);
   return !reuse;
+}
+
+// Whether this call's last CTA has cache state to update: a head whose entry is
+// still empty (it becomes valid), or the cumulative count (kept on every call).
+// Every thread of the CTA calls it; the result is CTA-uniform through the vote.
+__device__ __forceinline__ bool state_vote(const Params& p, int tid, int nthreads) {
+  int need = 0;
+  if (p.update_state) {
+    const int total = p.num_seqs * p.hq;
+    if ((p.flags & kGateTauCum) || total > 8 * nthreads) {
+      need = 1;
+    } else {
+      for (int i = tid; i < total; i += nthreads) need |= p.valid[i] == 0;
+    }
+  }
+  return __syncthreads_or(need) != 0;
+}
+
+// Cache-state epilogue: every CTA has read `valid` and `m_acc` (its decisions)
+// before it arrives on the completion counter; the last one to arrive marks the
+// heads that recomputed valid and advances the cumulative counts (0 after a
+// recompute, + n_updated after a reuse).  No CTA waits; the last one also resets
+// the counter for the next call.
+__device__ __forceinline__ void state_epilogue(const Params& p, int tid, int nthreads, int* s_flag) {
+  __syncthreads();
+  if (tid == 0) *s_flag = (atomicAdd(p.grid_ctr, 1) == static_cast<int>(gridDim.x) - 1) ? 1 : 0;
+  __syncthreads();
+  if (*s_flag) {
+    __threadfence();
+    const int total = p.num_seqs * p.hq;
+    for (int idx = tid; idx < total; idx += nthreads) {
+      const int b = idx / p.hq;
+      const bool rec = head_recompute(p, b, idx % p.hq);
+      if (rec) p.valid[idx] = 1;
+      if (p.flags & kGateTauCum) p.m_acc[idx] = rec ? 0 : p.m_acc[idx] + p.n_updated[b];
+    }
+    if (tid == 0) *p.grid_ctr = 0;
+  }
 }
 
 // Prefix chunks [a, b) of CTA s of S.  The last CTA also runs the `in_chunks`
@@ -380,17 +420,7 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   const int in0 = p.cu_in[b];
   const int n_in = p.cu_in[b + 1] - in0;
   if (tid < g) s_rec[tid] = head_recompute(p, b, hk * g + tid) ? 1 : 0;
-  // The cache-state epilogue only runs when some entry is still empty (valid = 0).
-  int invalid = 0;
-  if (p.update_state) {
-    const int total = p.num_seqs * p.hq;
-    if (total > 8 * C::kThreads) {
-      invalid = 1;
-    } else {
-      for (int i = tid; i < total; i += C::kThreads) invalid |= p.valid[i] == 0;
-    }
-  }
-  const bool need_state = __syncthreads_or(invalid) != 0;
+  const bool need_state = state_vote(p, tid, C::kThreads);
   const bool ranges_ok = q0 >= 0 && n_q >= 0 && q0 + n_q <= p.total_q && out0 >= 0 && n_out >= 0 &&
                          out0 + n_out <= p.total_out && in0 >= 0 && n_in >= 0 && in0 + n_in <= p.total_in &&
                          n_q <= n_in;
@@ -800,20 +830,7 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   }
 
   // ------------------------------------------------------------ cache-state epilogue
-  // Heads that recompute become valid.  Every CTA has read `valid` by now; the
-  // last one to arrive writes it (no CTA waits).
-  if (need_state) {
-    __syncthreads();
-    if (tid == 0) s_flag = (atomicAdd(p.grid_ctr, 1) == static_cast<int>(gridDim.x) - 1) ? 1 : 0;
-    __syncthreads();
-    if (s_flag) {
-      __threadfence();
-      const int total = p.num_seqs * p.hq;
-      for (int idx = tid; idx < total; idx += C::kThreads)
-        if (head_recompute(p, idx / p.hq, idx % p.hq)) p.valid[idx] = 1;
-      if (tid == 0) *p.grid_ctr = 0;
-    }
-  }
+  if (need_state) state_epilogue(p, tid, C::kThreads, &s_flag);
 }
 
 // ------------------------------------------------------------------ similarity gate
@@ -892,6 +909,69 @@ __global__ void __launch_bounds__(256) similarity_kernel(const SimParams p) {
     }
     const float den = sqrtf(sx) * sqrtf(sy);
     p.cos_out[blockIdx.x] = den > 0.f ? sd / den : 0.f;
+  }
+}
+
+// ------------------------------------------------------------------ branch hooks
+
+struct CacheCopyParams {
+  int hq, d, num_seqs, total_in, src, dst;
+  const int* cu_in;
+  float* a_out;
+  float* l_out;
+  uint8_t* valid;
+  __nv_bfloat16* q_ref;
+  int* m_acc;
+};
+
+// Entries of block positions 0..min(B_src, B_dst)-1 from sequence src to dst
+// (grid-stride over (position, head, 4 columns) items); block 0 also copies the
+// per-head validity and counts.
+__global__ void __launch_bounds__(256) cache_copy_kernel(const CacheCopyParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int s0 = p.cu_in[p.src], s1 = p.cu_in[p.src + 1];
+  const int d0 = p.cu_in[p.dst], d1 = p.cu_in[p.dst + 1];
+  if (s0 < 0 || s1 < s0 || s1 > p.total_in || d0 < 0 || d1 < d0 || d1 > p.total_in) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_status(kDevBadIndex);
+    return;
+  }
+  const int n = min(s1 - s0, d1 - d0);
+  const int c4 = p.d / 4;
+  const long items = static_cast<long>(n) * p.hq * c4;
+  for (long it = blockIdx.x * 256l + threadIdx.x; it < items; it += static_cast<long>(gridDim.x) * 256) {
+    const long e = it / c4;  // (position, head)
+    const int c = static_cast<int>(it % c4) * 4;
+    const long se = static_cast<long>(s0) * p.hq + e, de = static_cast<long>(d0) * p.hq + e;
+    *reinterpret_cast<float4*>(p.a_out + de * p.d + c) = *reinterpret_cast<const float4*>(p.a_out + se * p.d + c);
+    if (p.q_ref)
+      *reinterpret_cast<uint2*>(p.q_ref + de * p.d + c) = *reinterpret_cast<const uint2*>(p.q_ref + se * p.d + c);
+    if (c == 0) p.l_out[de] = p.l_out[se];
+  }
+  if (blockIdx.x == 0) {
+    const bool filled = d1 - d0 <= s1 - s0;
+    for (int h = threadIdx.x; h < p.hq; h += 256) {
+      p.valid[p.dst * p.hq + h] = filled ? p.valid[p.src * p.hq + h] : 0;
+      if (p.m_acc) p.m_acc[p.dst * p.hq + h] = p.m_acc[p.src * p.hq + h];
+    }
+  }
+}
+
+struct InvalidateParams {
+  int hq, num_seqs;
+  const uint8_t* mask;
+  uint8_t* valid;
+  int* m_acc;
+};
+
+__global__ void __launch_bounds__(256) cache_invalidate_kernel(const InvalidateParams p) {
+  pdl_wait();
+  pdl_trigger();
+  const int total = p.num_seqs * p.hq;
+  for (int i = blockIdx.x * 256 + threadIdx.x; i < total; i += gridDim.x * 256) {
+    if (p.mask && !p.mask[i / p.hq]) continue;
+    p.valid[i] = 0;
+    if (p.m_acc) p.m_acc[i] = 0;
   }
 }
 

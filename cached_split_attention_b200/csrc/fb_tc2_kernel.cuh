@@ -97,16 +97,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
   const int in0 = p.cu_in[b];
   const int n_in = p.cu_in[b + 1] - in0;
   if (tid == 0) s_rec0 = head_recompute(p, b, h) ? 1 : 0;
-  int invalid = 0;
-  {
-    const int total = p.num_seqs * p.hq;
-    if (total > 8 * kThreads) {
-      invalid = 1;
-    } else {
-      for (int i = tid; i < total; i += kThreads) invalid |= p.valid[i] == 0;
-    }
-  }
-  const bool need_state = __syncthreads_or(invalid) != 0;
+  const bool need_state = state_vote(p, tid, kThreads);
   const bool rec = s_rec0 != 0;
   const bool ranges_ok = q0 >= 0 && n_q >= 0 && q0 + n_q <= p.total_q && out0 >= 0 && n_out >= 0 &&
                          out0 + n_out <= p.total_out && in0 >= 0 && n_in >= 0 && in0 + n_in <= p.total_in &&
@@ -525,18 +516,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
   }
 
   // ------------------------------------------------------------ cache-state epilogue
-  if (need_state) {
-    __syncthreads();
-    if (tid == 0) s_flag = (atomicAdd(p.grid_ctr, 1) == static_cast<int>(gridDim.x) - 1) ? 1 : 0;
-    __syncthreads();
-    if (s_flag) {
-      __threadfence();
-      const int total = p.num_seqs * p.hq;
-      for (int idx = tid; idx < total; idx += kThreads)
-        if (head_recompute(p, idx / p.hq, idx % p.hq)) p.valid[idx] = 1;
-      if (tid == 0) *p.grid_ctr = 0;
-    }
-  }
+  if (need_state) state_epilogue(p, tid, kThreads, &s_flag);
 }
 
 }  // namespace fb

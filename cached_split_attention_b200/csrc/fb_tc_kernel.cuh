@@ -160,16 +160,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   const int in0 = p.cu_in[b];
   const int n_in = p.cu_in[b + 1] - in0;
   if (tid < g) s_rec[tid] = head_recompute(p, b, hk * g + tid) ? 1 : 0;
-  int invalid = 0;
-  if (p.update_state) {
-    const int total = p.num_seqs * p.hq;
-    if (total > 8 * kThreads) {
-      invalid = 1;
-    } else {
-      for (int i = tid; i < total; i += kThreads) invalid |= p.valid[i] == 0;
-    }
-  }
-  const bool need_state = __syncthreads_or(invalid) != 0;
+  const bool need_state = state_vote(p, tid, kThreads);
   const bool ranges_ok = q0 >= 0 && n_q >= 0 && q0 + n_q <= p.total_q && out0 >= 0 && n_out >= 0 &&
                          out0 + n_out <= p.total_out && in0 >= 0 && n_in >= 0 && in0 + n_in <= p.total_in &&
                          n_q <= n_in;
@@ -720,18 +711,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   }
 
   // ------------------------------------------------------------ cache-state epilogue
-  if (need_state) {
-    __syncthreads();
-    if (tid == 0) s_flag = (atomicAdd(p.grid_ctr, 1) == static_cast<int>(gridDim.x) - 1) ? 1 : 0;
-    __syncthreads();
-    if (s_flag) {
-      __threadfence();
-      const int total = p.num_seqs * p.hq;
-      for (int idx = tid; idx < total; idx += kThreads)
-        if (head_recompute(p, idx / p.hq, idx % p.hq)) p.valid[idx] = 1;
-      if (tid == 0) *p.grid_ctr = 0;
-    }
-  }
+  if (need_state) state_epilogue(p, tid, kThreads, &s_flag);
 }
 
 }  // namespace fb

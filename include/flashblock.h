@@ -65,6 +65,14 @@ typedef enum fb_status {
 #define FB_GATE_HEAD 2u       /* reuse head h only if cos(Q_bh, q_ref_bh) > gamma (strict) */
 #define FB_FORCE_RECOMPUTE 4u /* recompute every head (dense step)                        */
 #define FB_FORCE_REUSE 8u     /* reuse every head whose cache is valid                    */
+/* Cumulative threshold gate: reuse only if cache->m_acc[b,h] + n_updated[b] < tau, i.e.
+ * the block tokens updated since the head's cache was built (this step included) stay
+ * below tau; the count is kept in cache->m_acc and restarts at 0 when the head
+ * recomputes.  A reading of FlashBlock's updated-token count M ("Estrategias de
+ * Reutilizacion Adaptativa", first bullet), whose per-step form is FB_GATE_TAU; the two
+ * flags are exclusive.  The count is maintained on every call that sets the flag, forced
+ * modes and caller masks included. */
+#define FB_GATE_TAU_CUM 16u
 
 /*
  * One step's problem.  Index arrays are int32 device arrays; the scalar bounds
@@ -97,18 +105,21 @@ typedef struct fb_problem {
  *   valid [num_seqs, H_q] uint8 (0 = empty: the head recomputes whatever the gates say)
  *   q_ref [total_kv_in, H_q, d] bf16: the queries each head's entry was built with
  *         (needed by FB_GATE_HEAD; may be NULL otherwise)
+ *   m_acc [num_seqs, H_q] int32: block tokens updated since the head's last recompute
+ *         (needed by FB_GATE_TAU_CUM, zero-initialised by the caller; may be NULL otherwise)
  */
 typedef struct fb_cache {
   float* a_out;
   float* l_out;
   uint8_t* valid;
   fb_bf16* q_ref;
+  int32_t* m_acc;
 } fb_cache;
 
 typedef struct fb_params {
   int32_t tau;    /* threshold of FB_GATE_TAU */
   float gamma;    /* threshold of FB_GATE_HEAD */
-  uint32_t flags; /* FB_GATE_* | FB_FORCE_* */
+  uint32_t flags; /* FB_GATE_* | FB_FORCE_* (FB_GATE_TAU_CUM included) */
 } fb_params;
 
 /* Message of the last failing call on this thread (never NULL). */
@@ -194,6 +205,27 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
 /* Mark every cache entry of the problem's sequences empty (valid = 0): a new
  * block, a full refresh or a branch resync. */
 fb_status fb_cache_invalidate(const fb_problem* problem, const fb_cache* cache, fb_stream_t stream);
+
+/*
+ * Branch hooks for multi-branch decoding (BlockBatch, gist.science/fr/paper/2605.29233,
+ * "Methodologie : BlockBatch", items 2 and 3).  Both act on the FlashBlock cache only;
+ * the caller moves K/V itself.
+ *
+ * fb_cache_copy_seq -- leader-based synchronisation: the lagging branch dst_seq takes
+ *   the state of the leader src_seq.  For every q-head, the entries of block positions
+ *   0..min(B_src, B_dst)-1 (a_out, l_out, and q_ref / m_acc when present) are copied
+ *   from src_seq to dst_seq, and valid[dst_seq, :] = valid[src_seq, :]; when B_dst >
+ *   B_src the positions without a source leave dst_seq's heads empty (valid = 0).
+ *   src_seq == dst_seq is a no-op.  Errors: an index outside [0, num_seqs).
+ * fb_cache_invalidate_seqs -- periodic full-sequence refresh of some branches:
+ *   valid[b, :] = 0 (and m_acc[b, :] = 0 when present) for every b with
+ *   seq_mask[b] != 0 (uint8 [num_seqs], device); seq_mask NULL = every sequence.
+ * Asynchronous on `stream`; the problem's cu_seqlens_kv_in are read on the device.
+ */
+fb_status fb_cache_copy_seq(const fb_problem* problem, const fb_cache* cache, int32_t src_seq, int32_t dst_seq,
+                            fb_stream_t stream);
+fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* cache, const uint8_t* seq_mask,
+                                   fb_stream_t stream);
 
 /* Release the host-side tensor-map cache (descriptors of K/V buffers seen so far). */
 fb_status fb_release_cache(void);

@@ -51,12 +51,13 @@ def workspace_for(steps_problems, out_splits=0, device="cuda"):
     return ws
 
 
-def run_policy_gpu(w, flags=None, out_splits=0, head_reuse_in=None, device="cuda", keep=True):
-    """Run a workload's steps through fb_step; returns per-step dicts of numpy arrays."""
+def run_policy_gpu(w, flags=None, out_splits=0, head_reuse_in=None, device="cuda", keep=True, cache=None):
+    """Run a workload's steps through fb_step (on ``cache`` when given, else on a new
+    empty one); returns per-step dicts of numpy arrays and the cache."""
     torch, B = torch_and_binding()
     flags = w.flags if flags is None else flags
     p0 = w.problem
-    cache = B.Cache(p0, device, with_q_ref=True)
+    cache = cache if cache is not None else B.Cache(p0, device, with_q_ref=True)
     k_out = B.bf16_tensor(w.k_out, device)
     v_out = B.bf16_tensor(w.v_out, device)
     ws = workspace_for([st.problem for st in w.steps], out_splits, device)

@@ -76,6 +76,19 @@ def test_host_validation_without_gpu():
     rc = B._lib.fb_step(ctypes.byref(ok), ctypes.byref(prm), ctypes.byref(cache), 16, 16, 16, 16, 16, None, None,
                         16, 16, None, 16, 1 << 30, None)
     assert rc == B.ERR_INVALID_ARG and "n_updated" in B.last_error()
+    # the cumulative gate: exclusive with the per-step one, needs the count array
+    prm = B.params(4, 0.0, B.GATE_TAU | B.GATE_TAU_CUM)
+    rc = B._lib.fb_step(ctypes.byref(ok), ctypes.byref(prm), ctypes.byref(cache), 16, 16, 16, 16, 16, 16, None,
+                        16, 16, None, 16, 1 << 30, None)
+    assert rc == B.ERR_INVALID_ARG and "exclusive" in B.last_error()
+    prm = B.params(4, 0.0, B.GATE_TAU_CUM)
+    rc = B._lib.fb_step(ctypes.byref(ok), ctypes.byref(prm), ctypes.byref(cache), 16, 16, 16, 16, 16, 16, None,
+                        16, 16, None, 16, 1 << 30, None)
+    assert rc == B.ERR_INVALID_ARG and "m_acc" in B.last_error()
+    prm = B.params(4, 0.0, 32)
+    rc = B._lib.fb_step(ctypes.byref(ok), ctypes.byref(prm), ctypes.byref(cache), 16, 16, 16, 16, 16, 16, None,
+                        16, 16, None, 16, 1 << 30, None)
+    assert rc == B.ERR_INVALID_ARG and "unknown flag" in B.last_error()
     assert B._lib.fb_merge(-1, 4, 16, 16, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG
 
 

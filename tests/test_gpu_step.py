@@ -98,3 +98,56 @@ def test_two_tile_mha_locking():
     w = W.locking_tiny(steps=4, block=300, prefix=200, heads_q=2, heads_kv=2, head_dim=128)
     gpu, ref = _compare(w)
     assert any(r.recompute.any() and not r.recompute.all() for r in ref[1:]) or True
+
+
+def test_cumulative_tau_gate():
+    """FB_GATE_TAU_CUM: the updated tokens summed since each head's last recompute,
+    on the 8B-dLLM layer (full size): decisions bit-exact, outputs within tolerance,
+    and the device count equals the oracle's after the run."""
+    w = W.dllm_layer(steps=10)
+    gpu, cache = run_policy_gpu(w, flags=W.GATE_TAU_CUM)
+    ocache = policy.OracleCache.empty(w.problem)
+    ref = policy.run_policy(w, flags=W.GATE_TAU_CUM, cache=ocache)
+    for s, (g, r) in enumerate(zip(gpu, ref)):
+        assert np.array_equal(g["decision"], r.recompute), f"step {s}: decisions differ"
+        assert_close(g["a_full"], r.a_full, g["l_full"], r.l_full, f"cumulative step {s}")
+    recs = np.array([r.recompute[0, 0] for r in ref])
+    assert recs[0] and recs[1:].any() and not recs[1:].all()
+    assert np.array_equal(cache.m_acc.cpu().numpy()[:w.problem.num_seqs], ocache.m_acc)
+
+
+def test_branch_sync_and_refresh():
+    """BlockBatch hooks between steps of the varlen-branch workload: the 64-token
+    branch takes the 128-token leader's entries (leader sync), the 4-token branch is
+    refreshed.  The copy is bit-exact on the device; later steps match the oracle
+    applying the same hooks to its own cache."""
+    import dataclasses
+    import torch
+    from cached_split_attention_b200 import binding as B
+    w = W.varlen_branches(steps=4, prefix=512)
+    p0 = w.problem
+    first = dataclasses.replace(w, steps=w.steps[:2])
+    rest = dataclasses.replace(w, steps=w.steps[2:])
+    gpu, cache = run_policy_gpu(first)
+    ocache = policy.OracleCache.empty(p0)
+    policy.run_policy(first, cache=ocache)
+    dp = B.DeviceProblem(p0)
+    cu = p0.cu_seqlens_kv_in
+    src_rows = cache.a_out[cu[5]:cu[5] + (cu[5] - cu[4])].clone()
+    src_valid = cache.valid[5].clone()
+    mask = torch.zeros(p0.num_seqs, dtype=torch.uint8, device="cuda")
+    mask[0] = 1
+    B.cache_copy_seq(dp, cache, 5, 4)
+    B.cache_invalidate_seqs(dp, cache, mask)
+    torch.cuda.synchronize()
+    assert torch.equal(cache.a_out[cu[4]:cu[5]], src_rows)
+    assert torch.equal(cache.valid[4], src_valid) and not cache.valid[0].any()
+    policy.cache_copy_seq(ocache, p0, 5, 4)
+    policy.cache_invalidate_seqs(ocache, [b == 0 for b in range(p0.num_seqs)])
+    assert np.array_equal(cache.valid.cpu().numpy()[:p0.num_seqs].astype(bool), ocache.valid)
+    gpu2, _ = run_policy_gpu(rest, cache=cache)
+    ref2 = policy.run_policy(rest, cache=ocache)
+    for s, (g, r) in enumerate(zip(gpu2, ref2)):
+        assert np.array_equal(g["decision"], r.recompute), f"step {s + 2}: decisions differ"
+        assert_close(g["a_full"], r.a_full, g["l_full"], r.l_full, f"after hooks, step {s + 2}")
+    assert ref2[0].recompute[0].all()  # the refreshed branch recomputes
