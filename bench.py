@@ -22,9 +22,12 @@ over the K timed episodes (max over ranks).
 step's graph also copies every layer's block Q/K/V and update count from pinned
 host memory and copies A_full and L_full back.
 
-`roofline` is the fused attention kernel on its recompute launches (prefix pass +
-block pass + merge; HBM-bound), achieved = algorithmic bytes per launch / launch
-time on recompute steps; `roofline_all_launches` aggregates every launch.
+`roofline` is the attention kernel that serves the workload (KERNEL_OF) on its
+recompute launches (prefix pass + block pass + merge): HBM-bound workloads report
+algorithmic bytes per launch / launch time against the measured copy bandwidth,
+the video block (a dense contraction) algorithmic flops / time against the
+measured sustained bf16 tensor throughput; `roofline_all_launches` aggregates
+every launch.
 
 `--impl reference` times the fp64 oracle (the plain CPU statement of the method)
 on the host cores on one layer of the same workload, rank 0 only.
@@ -312,16 +315,28 @@ def _elapsed_us(ev):
     return np.array([[e0.elapsed_time(e1) * 1e3 for e0, e1 in row] for row in ev])
 
 
-def kernel_source_digest() -> str:
-    """sha256 over the CUDA sources of the attention path (the DRAM counters in
-    profiles/traffic.json are reported only while this digest matches)."""
+# The attention kernel that serves each workload's fused step (planned by
+# fb_api.cu: head_dim 128 with more than 64 rows per group -> tensor-core kernel,
+# multi-head with 256+ rows per head -> its two-tile form) and the sources it is
+# built from.
+KERNEL_OF = {"dllm_layer": "attn_kernel", "tiny": "attn_kernel", "long_context_gqa": "tc_attn_kernel",
+             "varlen_branches": "tc_attn_kernel", "video": "tc2_attn_kernel"}
+_BASE_SOURCES = ("fb_api.cu", "fb_device.cuh", "fb_kernels.cuh")
+KERNEL_SOURCES = {"attn_kernel": _BASE_SOURCES,
+                  "tc_attn_kernel": _BASE_SOURCES + ("fb_tcgen05.cuh", "fb_tc_kernel.cuh"),
+                  "tc2_attn_kernel": _BASE_SOURCES + ("fb_tcgen05.cuh", "fb_tc_kernel.cuh", "fb_tc2_kernel.cuh")}
+
+
+def kernel_source_digest(kernel: str = "attn_kernel") -> str:
+    """sha256 over the sources of one attention kernel (its code, device helpers and
+    the host planning that sizes its launch); the DRAM counters recorded for it in
+    profiles/traffic.json are reported only while this digest matches."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "cached_split_attention_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(name.encode())
-            h.update(open(os.path.join(csrc, name), "rb").read())
+    for name in KERNEL_SOURCES[kernel]:
+        h.update(name.encode())
+        h.update(open(os.path.join(csrc, name), "rb").read())
     return h.hexdigest()
 
 
@@ -408,14 +423,24 @@ def native(args, world, rank, local):
         pass
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    kernel = KERNEL_OF[args.workload]
     traffic = None
     try:
         prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-        # counters only count for the kernel source they were taken on
-        if prof.get("workload") == args.workload and prof.get("kernel_source_sha256") == kernel_source_digest():
-            traffic = prof.get("dram_bytes_per_recompute_launch")
+        for ent in prof.get("entries", []):
+            # counters only count for the kernel source they were taken on
+            if (ent.get("workload") == args.workload and ent.get("kernel") == kernel
+                    and ent.get("kernel_source_sha256") == kernel_source_digest(kernel)):
+                traffic = ent.get("dram_bytes_per_recompute_launch")
     except Exception:
         pass
+    # the video block is a dense contraction (about 1500 flop per byte): its bound
+    # is the tensor cores, timed inside a long step (the sustained bf16 figure)
+    tensor_bound = args.workload == "video"
+    flops_rec = [step_flops(w.steps[s].problem, rec_frac[s]) for s in rec_steps]
+    ach_tf = float(np.sum(flops_rec) / np.sum(t_rec) / 1e12) if rec_steps else float("nan")
+    tf_peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    tf_src = "measured, sustained" if "bf16_tflops_sustained" in peaks else "fallback, sustained"
 
     value = max_over_ranks(call_us, world, device)
     e2e_v = max_over_ranks(e2e_call_us, world, device)
@@ -457,17 +482,23 @@ def native(args, world, rank, local):
         "dense_call_us": {"median": round(dense_med, 3), "p10": round(float(np.percentile(dense_us, 10)), 3),
                           "p90": round(float(np.percentile(dense_us, 90)), 3),
                           "effective_tbps": round(dense_b / dense_med / 1e6, 3),
-                          "frac_of_hbm": round(dense_b / dense_med / 1e3 / hbm_peak, 4)},
+                          "frac_of_hbm": round(dense_b / dense_med / 1e3 / hbm_peak, 4),
+                          "tflops": round(step_flops(p, 1.0) / dense_med / 1e6, 1)},
         "reuse_call_us": {"median": round(reuse_med, 3), "p10": round(float(np.percentile(reuse_us, 10)), 3),
                           "p90": round(float(np.percentile(reuse_us, 90)), 3),
                           "effective_tbps": round(reuse_b / reuse_med / 1e6, 3)},
         "reuse_gain": {"predicted_bytes_ratio": round(dense_b / reuse_b, 2),
                        "achieved_time_ratio": round(dense_med / reuse_med, 2)},
-        "roofline": {"bound": "hbm", "kernel": "attn_kernel, recompute launches (prefix + block pass + merge)",
-                     "achieved": round(ach_rec, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(ach_rec / hbm_peak, 4), "peak_source": peak_src, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": round(float(np.mean(bytes_rec))) if rec_steps else None,
-                     "launches": len(rec_steps) * L * args.steps},
+        "roofline": dict(
+            ({"bound": "tensor", "achieved": round(ach_tf, 1), "peak": tf_peak, "unit": "TFLOP/s",
+              "frac": round(ach_tf / tf_peak, 4), "peak_source": tf_src, "hbm_gbs_achieved": round(ach_rec, 1)}
+             if tensor_bound else
+             {"bound": "hbm", "achieved": round(ach_rec, 1), "peak": hbm_peak, "unit": "GB/s",
+              "frac": round(ach_rec / hbm_peak, 4), "peak_source": peak_src}),
+            kernel=f"{kernel}, recompute launches (prefix + block pass + merge)", traffic=traffic,
+            algorithmic_bytes_per_launch=round(float(np.mean(bytes_rec))) if rec_steps else None,
+            algorithmic_flops_per_launch=round(float(np.mean(flops_rec))) if rec_steps else None,
+            launches=len(rec_steps) * L * args.steps),
         "roofline_all_launches": {"achieved": round(ach_all, 1), "unit": "GB/s",
                                   "frac": round(ach_all / hbm_peak, 4),
                                   "algorithmic_bytes_per_episode_per_layer": round(bytes_all)},
