@@ -262,3 +262,50 @@ def check_problem_vs_brute(attend_problem, merge, attend_full_fn=None, seed=4):
         af, lf = attend_full_fn(p, q, ko, vo, ki, vi)
         _close(af, np.array(ab), what="attend_full A")
         _close(lf, np.array(lb), what="attend_full L")
+
+
+def _sparse_case(seed=3):
+    """Two sequences (GQA 4/2, d = 16), prefixes 40 and 23, blocks 12 and 9 (a few
+    rows locked), bf16 inputs with sharp scores."""
+    from cached_split_attention_b200.workloads import make_problem, normal_bf16
+    rng = np.random.default_rng(seed)
+    p = make_problem([[0, 3, 4, 7, 11], [1, 2, 8]], [40, 23], [12, 9], 4, 2, 16)
+    q = normal_bf16(rng, (p.total_q, 4, 16), 0.6)
+    ko = normal_bf16(rng, (p.total_kv_out, 2, 16), 0.6)
+    vo = normal_bf16(rng, (p.total_kv_out, 2, 16))
+    ki = normal_bf16(rng, (p.total_kv_in, 2, 16), 0.6)
+    vi = normal_bf16(rng, (p.total_kv_in, 2, 16))
+    return p, q, ko, vo, ki, vi
+
+
+def check_sparse_partition(rearrange, attend_problem, attend_full, merge):
+    """The sparse-residual partition (FlashBlock, "Estrategias de Reutilizacion
+    Adaptativa", third bullet) is a partition of each sequence's keys: the rows of
+    J_out' and J_in' are those of prefix + block, once each; the block stays at
+    positions 0..B-1 of J_in'; with a fresh cache the merge of the two partials is
+    full attention over prefix + block; an empty selection changes nothing."""
+    p, q, ko, vo, ki, vi = _sparse_case()
+    for sel in ([[0, 5, 6, 39], [22]], [[], list(range(23))], [list(range(40)), []]):
+        p2, kr, vr, ke, ve = rearrange(p, ko, vo, ki, vi, sel)
+        for b in range(p.num_seqs):
+            orig = np.concatenate([ko[p.cu_seqlens_kv_out[b]:p.cu_seqlens_kv_out[b + 1]],
+                                   ki[p.cu_seqlens_kv_in[b]:p.cu_seqlens_kv_in[b + 1]]])
+            orig_v = np.concatenate([vo[p.cu_seqlens_kv_out[b]:p.cu_seqlens_kv_out[b + 1]],
+                                     vi[p.cu_seqlens_kv_in[b]:p.cu_seqlens_kv_in[b + 1]]])
+            new = np.concatenate([kr[p2.cu_seqlens_kv_out[b]:p2.cu_seqlens_kv_out[b + 1]],
+                                  ke[p2.cu_seqlens_kv_in[b]:p2.cu_seqlens_kv_in[b + 1]]])
+            new_v = np.concatenate([vr[p2.cu_seqlens_kv_out[b]:p2.cu_seqlens_kv_out[b + 1]],
+                                    ve[p2.cu_seqlens_kv_in[b]:p2.cu_seqlens_kv_in[b + 1]]])
+            key = lambda k, v: sorted(map(bytes, np.concatenate([k.reshape(len(k), -1), v.reshape(len(v), -1)], 1)))
+            assert key(orig, orig_v) == key(new, new_v), ("keys not a partition", b)
+            i0, i0n = int(p.cu_seqlens_kv_in[b]), int(p2.cu_seqlens_kv_in[b])
+            nb = int(p.cu_seqlens_kv_in[b + 1]) - i0
+            assert np.array_equal(ke[i0n:i0n + nb], ki[i0:i0 + nb]), ("block moved", b)
+        assert np.array_equal(p2.q_rows, p.q_rows) and np.array_equal(p2.cu_seqlens_q, p.cu_seqlens_q)
+        a_o, l_o = attend_problem(p2, q, kr, vr, "out")
+        a_i, l_i = attend_problem(p2, q, ke, ve, "in")
+        a, l = merge(a_o, l_o, a_i, l_i)
+        a_ex, l_ex = attend_full(p, q, ko, vo, ki, vi)
+        assert np.abs(a - a_ex).max() < 1e-12 and np.abs(l - l_ex).max() < 1e-12, "fresh partition is not exact"
+    p2, kr, vr, ke, ve = rearrange(p, ko, vo, ki, vi, [[], []])
+    assert np.array_equal(kr, ko) and np.array_equal(ve, vi) and np.array_equal(p2.cu_seqlens_kv_in, p.cu_seqlens_kv_in)

@@ -145,3 +145,21 @@ def test_unmutated_oracle_passes_every_pin():
     pins.check_golden_gates(policy.decide)
     pins.check_cosine(policy.head_cosine)
     pins.check_problem_vs_brute(attention.attend_problem, attention.merge)
+
+
+SPARSE_MUTANTS = [
+    ("selected keys also left in the residual", "keep[sel] = False", "keep[sel] = keep[sel]"),
+    ("selected keys dropped", "ext_k.append(np.concatenate([k_in[i0:i1], k_out[o0:o1][sel]]))",
+     "ext_k.append(np.concatenate([k_in[i0:i1], k_out[o0:o1][sel][:0]]))"),
+    ("selection placed before the block", "ext_k.append(np.concatenate([k_in[i0:i1], k_out[o0:o1][sel]]))",
+     "ext_k.append(np.concatenate([k_out[o0:o1][sel], k_in[i0:i1]]))"),
+    ("values gathered from the keys", "res_v.append(v_out[o0:o1][keep])", "res_v.append(k_out[o0:o1][keep])"),
+]
+
+
+@pytest.mark.parametrize("label,old,new", SPARSE_MUTANTS, ids=[m[0] for m in SPARSE_MUTANTS])
+def test_sparse_mutants_caught(label, old, new):
+    from oracle import sparse
+    bad = mutate(sparse, "rearrange", old, new)
+    assert caught(pins.check_sparse_partition, bad, attention.attend_problem, attention.attend_full,
+                  attention.merge), label
