@@ -321,16 +321,16 @@ def _elapsed_us(ev):
 # built from.
 KERNEL_OF = {"dllm_layer": "attn_kernel", "tiny": "attn_kernel", "long_context_gqa": "tc_attn_kernel",
              "varlen_branches": "tc_attn_kernel", "video": "tc2_attn_kernel"}
-_BASE_SOURCES = ("fb_api.cu", "fb_device.cuh", "fb_kernels.cuh")
+_BASE_SOURCES = ("fb_device.cuh", "fb_kernels.cuh")
 KERNEL_SOURCES = {"attn_kernel": _BASE_SOURCES,
                   "tc_attn_kernel": _BASE_SOURCES + ("fb_tcgen05.cuh", "fb_tc_kernel.cuh"),
                   "tc2_attn_kernel": _BASE_SOURCES + ("fb_tcgen05.cuh", "fb_tc_kernel.cuh", "fb_tc2_kernel.cuh")}
 
 
 def kernel_source_digest(kernel: str = "attn_kernel") -> str:
-    """sha256 over the sources of one attention kernel (its code, device helpers and
-    the host planning that sizes its launch); the DRAM counters recorded for it in
-    profiles/traffic.json are reported only while this digest matches."""
+    """sha256 over the device sources of one attention kernel (its code and device
+    helpers); the DRAM counters recorded for it in profiles/traffic.json are
+    reported only while this digest matches."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "cached_split_attention_b200", "csrc")
