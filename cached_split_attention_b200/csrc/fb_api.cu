@@ -12,6 +12,7 @@
 #include <string>
 #include <unordered_map>
 
+#include "fb_sparse.cuh"
 #include "fb_tc2_kernel.cuh"
 #include "flashblock.h"
 
@@ -553,6 +554,51 @@ fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* ca
   const int blocks = std::min((total + 255) / 256, 148);
   cudaError_t e = launch_pdl(fb::cache_invalidate_kernel, blocks, 256, reinterpret_cast<cudaStream_t>(stream), ip);
   if (e != cudaSuccess) return cuda_fail(e, "cache invalidate kernel launch");
+  return FB_OK;
+}
+
+fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, const int32_t* sel_idx,
+                           int32_t total_sel, const fb_bf16* k_out, const fb_bf16* v_out, const fb_bf16* k_in,
+                           const fb_bf16* v_in, fb_bf16* k_res, fb_bf16* v_res, fb_bf16* k_ext, fb_bf16* v_ext,
+                           int32_t* cu_seqlens_kv_out_res, int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  if (total_sel < 0 || total_sel > problem->total_kv_out)
+    return fail(FB_ERR_INVALID_ARG, "total_sel %d outside [0, total_kv_out]", total_sel);
+  if (problem->num_seqs == 0) return FB_OK;
+  if (!cu_sel) return fail(FB_ERR_INVALID_ARG, "cu_sel is NULL");
+  if (total_sel > 0 && !sel_idx) return fail(FB_ERR_INVALID_ARG, "sel_idx is NULL");
+  const bool res = problem->total_kv_out - total_sel > 0;
+  const bool ext = problem->total_kv_in + total_sel > 0;
+  FB_TRY(check_ptr(k_out, "k_out", problem->total_kv_out > 0));
+  FB_TRY(check_ptr(v_out, "v_out", problem->total_kv_out > 0));
+  FB_TRY(check_ptr(k_in, "k_in", problem->total_kv_in > 0));
+  FB_TRY(check_ptr(v_in, "v_in", problem->total_kv_in > 0));
+  FB_TRY(check_ptr(k_res, "k_res", res));
+  FB_TRY(check_ptr(v_res, "v_res", res));
+  FB_TRY(check_ptr(k_ext, "k_ext", ext));
+  FB_TRY(check_ptr(v_ext, "v_ext", ext));
+  fb::SparseParams sp{problem->num_seqs, problem->num_heads_kv, problem->head_dim, problem->total_kv_out,
+                      problem->total_kv_in, total_sel, problem->cu_seqlens_kv_out, problem->cu_seqlens_kv_in, cu_sel,
+                      sel_idx, reinterpret_cast<const __nv_bfloat16*>(k_out),
+                      reinterpret_cast<const __nv_bfloat16*>(v_out), reinterpret_cast<const __nv_bfloat16*>(k_in),
+                      reinterpret_cast<const __nv_bfloat16*>(v_in), reinterpret_cast<__nv_bfloat16*>(k_res),
+                      reinterpret_cast<__nv_bfloat16*>(v_res), reinterpret_cast<__nv_bfloat16*>(k_ext),
+                      reinterpret_cast<__nv_bfloat16*>(v_ext), cu_seqlens_kv_out_res, cu_seqlens_kv_in_ext};
+  const long per_seq = static_cast<long>(problem->max_kv_out + problem->max_kv_in) * problem->num_heads_kv *
+                       problem->head_dim / 8;
+  const int bx = static_cast<int>(std::max<long>(1, std::min<long>((per_seq + 255) / 256, 256)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(bx, problem->num_seqs);
+  cfg.blockDim = dim3(256);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[] = {&sp};
+  cudaError_t e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&fb::sparse_layout_kernel), args);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse layout kernel launch");
   return FB_OK;
 }
 

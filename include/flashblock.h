@@ -227,6 +227,33 @@ fb_status fb_cache_copy_seq(const fb_problem* problem, const fb_cache* cache, in
 fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* cache, const uint8_t* seq_mask,
                                    fb_stream_t stream);
 
+/*
+ * Sparse-residual layout (FlashBlock, gist.science/es/paper/2602.05305, "Estrategias de
+ * Reutilizacion Adaptativa", third bullet: the keys a sparse-attention pattern does not
+ * select form the out-of-block set, whose contribution FlashBlock caches).  For every
+ * sequence b the selected prefix keys join the block's keys and the rest form the
+ * residual prefix:
+ *   J_in'(b)  = block keys of b, then the selected prefix keys (increasing order)
+ *   J_out'(b) = prefix keys of b that are not selected (order kept)
+ * cu_sel [num_seqs+1] (device) offsets into sel_idx; sel_idx [total_sel] (device) holds,
+ * per sequence, strictly increasing positions in [0, N_b) of the selected prefix keys;
+ * total_sel (host) = cu_sel[num_seqs].  Outputs (device, THD bf16, caller-owned):
+ *   k_res, v_res [total_kv_out - total_sel, H_kv, d];  k_ext, v_ext [total_kv_in + total_sel, H_kv, d]
+ *   cu_seqlens_kv_out_res = cu_seqlens_kv_out - cu_sel, cu_seqlens_kv_in_ext =
+ *   cu_seqlens_kv_in + cu_sel ([num_seqs+1] each; may be NULL).
+ * The block keeps positions 0..B_b-1 of J_in', so cu_seqlens_q and q_rows stay valid:
+ * fb_step on (J_out', J_in') with a cache of total_kv_in + total_sel rows caches the
+ * residual and recomputes the selected keys every step; with a fresh cache the result is
+ * full attention over prefix and block.  The selection is fixed for a block (a new one
+ * changes the residual: refill the cache).  A selection that is not increasing or out of
+ * range records FB_ERR_INVALID_ARG on the device (fb_device_status); that sequence is
+ * skipped.
+ */
+fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, const int32_t* sel_idx,
+                           int32_t total_sel, const fb_bf16* k_out, const fb_bf16* v_out, const fb_bf16* k_in,
+                           const fb_bf16* v_in, fb_bf16* k_res, fb_bf16* v_res, fb_bf16* k_ext, fb_bf16* v_ext,
+                           int32_t* cu_seqlens_kv_out_res, int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream);
+
 /* Release the host-side tensor-map cache (descriptors of K/V buffers seen so far). */
 fb_status fb_release_cache(void);
 
