@@ -350,29 +350,40 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
         }
         tc_fence_after();  // S(c) done, and with it every earlier MMA (PV(c-1) included)
         if (rec && c == nB && nB > 0) snapshot();
-        // row max of the raw scores (the whole S row in one TMEM round trip)
+        // row max of the raw scores (the whole S row in one TMEM round trip); the
+        // first 64 columns stay in registers for the exponentials
         float mxa[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+        uint32_t sk[2][32];
         {
-          uint32_t sv[4][32];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) tmem_ld32(sp + 32 * i, sv[i]);
+          uint32_t sv[2][32];
+          tmem_ld32(sp, sk[0]);
+          tmem_ld32(sp + 32, sk[1]);
+          tmem_ld32(sp + 64, sv[0]);
+          tmem_ld32(sp + 96, sv[1]);
           tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 4; ++i) reg_fence32(sv[i]);
+          reg_fence32(sk[0]);
+          reg_fence32(sk[1]);
+          reg_fence32(sv[0]);
+          reg_fence32(sv[1]);
           if (valid < kN) {  // ragged last chunk of a segment
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 2; ++i) {
 #pragma unroll
-              for (int k = 0; k < 32; ++k)
-                if (32 * i + k >= valid) sv[i][k] = __float_as_uint(kNegInf);
+              for (int k = 0; k < 32; ++k) {
+                if (32 * i + k >= valid) sk[i][k] = __float_as_uint(kNegInf);
+                if (64 + 32 * i + k >= valid) sv[i][k] = __float_as_uint(kNegInf);
+              }
             }
           }
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < 2; ++i) {
 #pragma unroll
-            for (int k = 0; k < 32; k += 2)
+            for (int k = 0; k < 32; k += 2) {
+              mxa[(k >> 1) & 3] =
+                  tc::max3(mxa[(k >> 1) & 3], __uint_as_float(sk[i][k]), __uint_as_float(sk[i][k + 1]));
               mxa[(k >> 1) & 3] =
                   tc::max3(mxa[(k >> 1) & 3], __uint_as_float(sv[i][k]), __uint_as_float(sv[i][k + 1]));
+            }
           }
         }
         const float mx = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])) * p.scale_log2;
@@ -399,44 +410,47 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
           }
         }
         const uint64_t nm2 = f2_pack(m == kNegInf ? 0.f : -m, m == kNegInf ? 0.f : -m);
-        // P = 2^(s * scale - m), two 64-column halves (one TMEM round trip each),
-        // each 32-column group stored over its S columns
+        // P = 2^(s * scale - m): the kept first half while the second half comes
+        // back from TMEM; each 32-column group of P is stored over S columns whose
+        // scores are already in registers
         uint64_t rsa[2] = {0ull, 0ull};
+        auto exp_group = [&](const uint32_t (&sg)[32], uint32_t col) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          uint32_t sv[2][32];
-          tmem_ld32(sp + 64 * hlf, sv[0]);
-          tmem_ld32(sp + 64 * hlf + 32, sv[1]);
-          tmem_wait_ld();
-          reg_fence32(sv[0]);
-          reg_fence32(sv[1]);
+          for (int k = 0; k < 32; k += 2) {
+            const uint64_t xx = ffma2(f2_pack(__uint_as_float(sg[k]), __uint_as_float(sg[k + 1])), scale2, nm2);
+            float p0, p1;
+            if (((k >> 1) & 7) < 3) {
+              tc::exp2_poly2(xx, p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(xx, x0, x1);
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            rsa[(k >> 1) & 1] = fadd2(rsa[(k >> 1) & 1], f2_pack(p0, p1));
+            pk[k >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(sp + col, pk);
+        };
+        uint32_t sh[2][32];
+        tmem_ld32(sp + 64, sh[0]);
+        tmem_ld32(sp + 96, sh[1]);
+        exp_group(sk[0], 0);
+        exp_group(sk[1], 16);
+        tmem_wait_ld();
+        reg_fence32(sh[0]);
+        reg_fence32(sh[1]);
+        if (valid < kN) {
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
-            if (valid < kN) {
 #pragma unroll
-              for (int k = 0; k < 32; ++k)
-                if (64 * hlf + 32 * i + k >= valid) sv[i][k] = __float_as_uint(kNegInf);
-            }
-            uint32_t pk[16];
-#pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              const uint64_t xx =
-                  ffma2(f2_pack(__uint_as_float(sv[i][k]), __uint_as_float(sv[i][k + 1])), scale2, nm2);
-              float p0, p1;
-              if (((k >> 1) & 7) < 3) {
-                tc::exp2_poly2(xx, p0, p1);
-              } else {
-                float x0, x1;
-                f2_unpack(xx, x0, x1);
-                p0 = ex2(x0);
-                p1 = ex2(x1);
-              }
-              rsa[(k >> 1) & 1] = fadd2(rsa[(k >> 1) & 1], f2_pack(p0, p1));
-              pk[k >> 1] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16(sp + 32 * hlf + 16 * i, pk);
+            for (int k = 0; k < 32; ++k)
+              if (64 + 32 * i + k >= valid) sh[i][k] = __float_as_uint(kNegInf);
           }
         }
+        exp_group(sh[0], 32);
+        exp_group(sh[1], 48);
         float r0, r1, r2, r3;
         f2_unpack(rsa[0], r0, r1);
         f2_unpack(rsa[1], r2, r3);
