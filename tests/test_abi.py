@@ -90,6 +90,15 @@ def test_host_validation_without_gpu():
                         16, 16, None, 16, 1 << 30, None)
     assert rc == B.ERR_INVALID_ARG and "unknown flag" in B.last_error()
     assert B._lib.fb_merge(-1, 4, 16, 16, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG
+    # branch hooks and the sparse layout: argument checks before any device work
+    cache5 = B.FbCache(16, 16, 16, 0, 0)
+    assert B._lib.fb_cache_copy_seq(ctypes.byref(ok), ctypes.byref(cache5), 0, 3, None) == B.ERR_INVALID_ARG
+    assert "out of range" in B.last_error()
+    assert B._lib.fb_cache_copy_seq(ctypes.byref(ok), ctypes.byref(cache5), 0, 0, None) == B.OK  # no-op
+    rc = B._lib.fb_sparse_layout(ctypes.byref(ok), 16, 16, 5000, 16, 16, 16, 16, 16, 16, 16, 16, None, None, None)
+    assert rc == B.ERR_INVALID_ARG and "total_sel" in B.last_error()
+    rc = B._lib.fb_sparse_layout(ctypes.byref(ok), None, 16, 4, 16, 16, 16, 16, 16, 16, 16, 16, None, None, None)
+    assert rc == B.ERR_INVALID_ARG and "cu_sel" in B.last_error()
 
 
 def test_workspace_size_is_counter_plus_scores():
