@@ -12,6 +12,7 @@
 #include <string>
 #include <unordered_map>
 
+#include "fb_order.cuh"
 #include "fb_sparse.cuh"
 #include "fb_tc2_kernel.cuh"
 #include "flashblock.h"
@@ -85,7 +86,8 @@ struct Plan {
   bool tc = false;   // tensor-core kernel (tcgen05): head_dim 128, more than 64 rows per group
   bool tc2 = false;  // two-tile tensor-core kernel: fused step, MHA, at least 256 rows per head
   int bn = fb::kBN;  // keys per pipeline chunk (TMA box rows)
-  size_t off_grid_ctr = 0, off_cos = 0, bytes = 0;
+  size_t off_grid_ctr = 0, off_cos = 0, off_order = 0, bytes = 0;
+  int order_items = 0;  // work items of the two-tile kernel (0: the problem never takes it)
 };
 
 int device_sms() {
@@ -187,6 +189,12 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = fals
   off = align_up(off + sizeof(int), 256);
   pl.off_cos = off;
   off = align_up(off + sizeof(float) * std::max(1, p->num_seqs * p->num_heads_q), 256);
+  // work order of the two-tile kernel, for every problem that fb_step may give it
+  if (pl.d == 128 && pl.g == 1 && p->max_q >= 2 * fb::tc2::kM) {
+    pl.order_items = p->num_seqs * p->num_heads_q * ((p->max_q + 2 * fb::tc2::kM - 1) / (2 * fb::tc2::kM));
+    pl.off_order = off;
+    off = align_up(off + sizeof(int) * pl.order_items, 256);
+  }
   pl.bytes = off;
   return pl;
 }
@@ -293,8 +301,8 @@ fb_status launch_attn(const Plan& pl, fb::Params& prm, cudaStream_t stream) {
 
 // Launch of a kernel without clusters, allowed to start while the previous
 // kernel of the stream finishes (each kernel waits for it before reading).
-template <typename Arg>
-cudaError_t launch_pdl(void (*fn)(Arg), int blocks, int threads, cudaStream_t stream, const Arg& arg) {
+template <typename... Args>
+cudaError_t launch_pdl(void (*fn)(Args...), int blocks, int threads, cudaStream_t stream, const Args&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(threads);
@@ -304,9 +312,8 @@ cudaError_t launch_pdl(void (*fn)(Arg), int blocks, int threads, cudaStream_t st
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  Arg a = arg;
-  void* args[] = {&a};
-  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(fn), args);
+  void* argv[] = {const_cast<void*>(static_cast<const void*>(&args))...};  // copied at launch
+  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(fn), argv);
 }
 
 void fill_problem(const fb_problem* p, const Plan& pl, fb::Params& prm) {
@@ -491,6 +498,7 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
     float* cos_ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_cos);
     FB_TRY(fb_head_similarity(problem, q, cache->q_ref, cos_ws, stream));
   }
+  const bool order_work = pl.tc2 && uses_gates && rows;  // decisions may differ per head
   prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
   prm.do_out = 1;
   prm.do_in = 1;
@@ -509,6 +517,15 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   prm.a_full = reinterpret_cast<__nv_bfloat16*>(a_full);
   prm.l_full = l_full;
   prm.decision_out = decision_out;
+  if (order_work) {
+    int* order = reinterpret_cast<int*>(static_cast<char*>(workspace) + pl.off_order);
+    if (pl.n_groups != pl.order_items)
+      return fail(FB_ERR_INVALID_ARG, "internal: %d work items, order sized for %d", pl.n_groups, pl.order_items);
+    int* order_arg = order;
+    cudaError_t e = launch_pdl(fb::order_kernel, 1, fb::kOrderThreads, st, prm, order_arg);
+    if (e != cudaSuccess) return cuda_fail(e, "order kernel launch");
+    prm.order = order;
+  }
   return launch_attn(pl, prm, st);
 }
 

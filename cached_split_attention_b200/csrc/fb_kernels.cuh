@@ -85,7 +85,8 @@ struct alignas(64) Params {
   float* a_in;
   float* l_in;
   // workspace
-  int* grid_ctr;  // completion counter of the cache-state epilogue (zero between calls)
+  int* grid_ctr;     // completion counter of the cache-state epilogue (zero between calls)
+  const int* order;  // work order of the two-tile kernel (NULL: CTA i takes item i)
 };
 
 // Reuse decision of (b, h); see fb_step in flashblock.h.

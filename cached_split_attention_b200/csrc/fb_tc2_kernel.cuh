@@ -85,9 +85,10 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int pair = blockIdx.x % p.tiles;  // p.tiles counts 256-row pairs here
-  const int h = blockIdx.x / p.tiles % p.hq;
-  const int b = blockIdx.x / p.tiles / p.hq;
+  const int item = p.order ? p.order[blockIdx.x] : static_cast<int>(blockIdx.x);  // (b, h, pair)
+  const int pair = item % p.tiles;  // p.tiles counts 256-row pairs here
+  const int h = item / p.tiles % p.hq;
+  const int b = item / p.tiles / p.hq;
 
   // ------------------------------------------------------------ metadata
   const int q0 = p.cu_q[b];

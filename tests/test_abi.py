@@ -111,3 +111,10 @@ def test_workspace_size_is_counter_plus_scores():
         prob = _problem(B, num_seqs=seqs, num_heads_q=hq, num_heads_kv=hq, out_splits=4)
         assert B._lib.fb_workspace_size(ctypes.byref(prob), ctypes.byref(n)) == B.OK
         assert n.value == expect, (seqs, hq, n.value)
+    # a multi-head problem of 256+ rows per head may take the two-tile kernel: its
+    # work order (one int32 per (sequence, head, 256-row pair)) follows
+    n = ctypes.c_size_t()
+    prob = _problem(B, num_heads_q=40, num_heads_kv=40, total_q=1560, max_q=1560, total_kv_in=1560,
+                    max_kv_in=1560)
+    assert B._lib.fb_workspace_size(ctypes.byref(prob), ctypes.byref(n)) == B.OK
+    assert n.value == 256 + 256 + 1280, n.value  # 40 x 7 items x 4 bytes = 1120 -> 1280
