@@ -72,6 +72,7 @@ def _load():
         "fb_cache_copy_seq": (st, [P, ctypes.POINTER(FbCache), ctypes.c_int32, ctypes.c_int32, vp]),
         "fb_cache_invalidate_seqs": (st, [P, ctypes.POINTER(FbCache), vp, vp]),
         "fb_sparse_layout": (st, [P, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "fb_selftest_wait_timeout": (st, [vp]),
         "fb_release_cache": (st, []),
         "fb_device_status": (st, [ctypes.POINTER(ctypes.c_int32), vp]),
         "fb_step_noalloc": (st, [P, ctypes.POINTER(FbParams), ctypes.POINTER(FbCache), vp, vp, vp, vp, vp, vp, vp,
@@ -241,6 +242,10 @@ def sparse_layout(problem: DeviceProblem, cu_sel, sel_idx, total_sel: int, k_out
     _check(_lib.fb_sparse_layout(problem.ref, _ptr(cu_sel), _ptr(sel_idx), int(total_sel), _ptr(k_out), _ptr(v_out),
                                  _ptr(k_in), _ptr(v_in), _ptr(k_res), _ptr(v_res), _ptr(k_ext), _ptr(v_ext),
                                  _ptr(cu_out_res), _ptr(cu_in_ext), _stream(stream)))
+
+
+def selftest_wait_timeout(stream=None):
+    _check(_lib.fb_selftest_wait_timeout(_stream(stream)))
 
 
 def release_cache():

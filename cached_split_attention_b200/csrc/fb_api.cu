@@ -13,6 +13,7 @@
 #include <unordered_map>
 
 #include "fb_order.cuh"
+#include "fb_selftest.cuh"
 #include "fb_sparse.cuh"
 #include "fb_tc2_kernel.cuh"
 #include "flashblock.h"
@@ -616,6 +617,13 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
   void* args[] = {&sp};
   cudaError_t e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&fb::sparse_layout_kernel), args);
   if (e != cudaSuccess) return cuda_fail(e, "sparse layout kernel launch");
+  return FB_OK;
+}
+
+fb_status fb_selftest_wait_timeout(fb_stream_t stream) {
+  fb::wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "self-test kernel launch");
   return FB_OK;
 }
 

@@ -254,6 +254,15 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
                            const fb_bf16* v_in, fb_bf16* k_res, fb_bf16* v_res, fb_bf16* k_ext, fb_bf16* v_ext,
                            int32_t* cu_seqlens_kv_out_res, int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream);
 
+/*
+ * Self-test of the failure path of the bounded waits (no counterpart in the pages):
+ * launches one CTA that waits on an mbarrier nothing will ever complete, with the same
+ * bounded wait the attention kernels use (about two seconds), so the wait runs out,
+ * FB_ERR_TIMEOUT is recorded in the device status word and the kernel returns; the
+ * context stays usable.  Read the result with fb_device_status().
+ */
+fb_status fb_selftest_wait_timeout(fb_stream_t stream);
+
 /* Release the host-side tensor-map cache (descriptors of K/V buffers seen so far). */
 fb_status fb_release_cache(void);
 
