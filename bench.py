@@ -20,7 +20,8 @@ over the K timed episodes (max over ranks).
 
 `e2e` is the same metric through the public API with host buffers: each denoise
 step's graph also copies every layer's block Q/K/V and update count from pinned
-host memory and copies A_full and L_full back.
+host memory and copies A_full and L_full back, on two copy streams that overlap
+the uploads and downloads with the other layers' attention.
 
 `roofline` is the attention kernel that serves the workload (KERNEL_OF) on its
 recompute launches (prefix pass + block pass + merge): HBM-bound workloads report
@@ -208,58 +209,96 @@ class Model:
         self.dp = [B.DeviceProblem(st.problem, device) for st in w.steps]
         wsz = max(B.workspace_size(d) for d in self.dp)
         k_out0, v_out0 = B.bf16_tensor(w.k_out, device), B.bf16_tensor(w.v_out, device)
-        q0 = [B.bf16_tensor(st.q, device) for st in w.steps]
-        ki0 = [B.bf16_tensor(st.k_in, device) for st in w.steps]
-        vi0 = [B.bf16_tensor(st.v_in, device) for st in w.steps]
-        n0 = [torch.as_tensor(st.n_updated, dtype=torch.int32).to(device) for st in w.steps]
         H, d = p.num_heads_q, p.head_dim
         tq = max(st.problem.total_q for st in w.steps)
+        # Each step's block inputs of a layer live in one device blob (Q, K_in, V_in,
+        # n_updated at 256-byte aligned offsets) and the outputs in another (A_full,
+        # L_full), so the end-to-end leg moves each with a single copy; the pinned
+        # host blobs have the same layout (the inputs are shared by the layers).
+        self.in_layout = []
+        host_in = []
+        for st in w.steps:
+            parts = [st.q.view(np.uint8).reshape(-1), st.k_in.view(np.uint8).reshape(-1),
+                     st.v_in.view(np.uint8).reshape(-1), st.n_updated.astype(np.int32).view(np.uint8)]
+            offs, off = [], 0
+            for a in parts:
+                offs.append(off)
+                off = (off + a.nbytes + 255) // 256 * 256
+            blob = np.zeros(off, dtype=np.uint8)
+            for o, a in zip(offs, parts):
+                blob[o:o + a.nbytes] = a
+            self.in_layout.append((offs, [a.nbytes for a in parts], st.q.shape, st.k_in.shape))
+            host_in.append(blob)
+        a_bytes = (tq * H * d * 2 + 255) // 256 * 256
+        self.out_bytes = a_bytes + tq * H * 4
         self.layers = []
         for _ in range(layers):
-            lay = dict(
-                k_out=k_out0.clone(), v_out=v_out0.clone(),
-                q=[x.clone() for x in q0], k_in=[x.clone() for x in ki0], v_in=[x.clone() for x in vi0],
-                n=[x.clone() for x in n0],
-                cache=B.Cache(p, device, with_q_ref=bool(w.flags & W.GATE_HEAD)),
-                ws=torch.empty(wsz, dtype=torch.uint8, device=device),
-                a_full=torch.empty((tq, H, d), dtype=torch.bfloat16, device=device),
-                l_full=torch.empty((tq, H), dtype=torch.float32, device=device),
-                dec=torch.empty((p.num_seqs, H), dtype=torch.uint8, device=device))
+            lay = dict(k_out=k_out0.clone(), v_out=v_out0.clone(), inb=[], q=[], k_in=[], v_in=[], n=[],
+                       cache=B.Cache(p, device, with_q_ref=bool(w.flags & W.GATE_HEAD)),
+                       ws=torch.empty(wsz, dtype=torch.uint8, device=device),
+                       outb=torch.empty(self.out_bytes, dtype=torch.uint8, device=device),
+                       dec=torch.empty((p.num_seqs, H), dtype=torch.uint8, device=device))
+            for s_, blob in enumerate(host_in):
+                offs, sizes, qshape, kshape = self.in_layout[s_]
+                dblob = torch.from_numpy(blob).to(device)
+                lay["inb"].append(dblob)
+                lay["q"].append(dblob[offs[0]:offs[0] + sizes[0]].view(torch.bfloat16).view(qshape))
+                lay["k_in"].append(dblob[offs[1]:offs[1] + sizes[1]].view(torch.bfloat16).view(kshape))
+                lay["v_in"].append(dblob[offs[2]:offs[2] + sizes[2]].view(torch.bfloat16).view(kshape))
+                lay["n"].append(dblob[offs[3]:offs[3] + sizes[3]].view(torch.int32))
+            lay["a_full"] = lay["outb"][:tq * H * d * 2].view(torch.bfloat16).view(tq, H, d)
+            lay["l_full"] = lay["outb"][a_bytes:a_bytes + tq * H * 4].view(torch.float32).view(tq, H)
             B.workspace_init(lay["ws"])
             self.layers.append(lay)
-        del k_out0, v_out0, q0, ki0, vi0, n0
-        # pinned host copies for the end-to-end leg (shared by the layers)
-        self.h_q = [torch.from_numpy(st.q.view(np.int16)).pin_memory() for st in w.steps]
-        self.h_k = [torch.from_numpy(st.k_in.view(np.int16)).pin_memory() for st in w.steps]
-        self.h_v = [torch.from_numpy(st.v_in.view(np.int16)).pin_memory() for st in w.steps]
-        self.h_n = [torch.from_numpy(st.n_updated.astype(np.int32)).pin_memory() for st in w.steps]
-        self.h_a = [torch.empty((tq, H, d), dtype=torch.bfloat16).pin_memory() for _ in range(layers)]
-        self.h_l = [torch.empty((tq, H), dtype=torch.float32).pin_memory() for _ in range(layers)]
+        del k_out0, v_out0
+        self.h_in = [torch.from_numpy(b).pin_memory() for b in host_in]
+        self.h_out = [torch.empty(self.out_bytes, dtype=torch.uint8).pin_memory() for _ in range(layers)]
         # L2 flush: read 256 MiB (about twice the L2)
         self.flush_buf = torch.ones(64 << 20, dtype=torch.int32, device=device)
         self.flush_out = torch.empty((), dtype=torch.int32, device=device)
         self.graphs = {}
+        # end-to-end leg: inputs come in on one copy stream, results leave on
+        # another, so layer l+1's upload and layer l-1's download overlap layer l
+        self.copy_in = torch.cuda.Stream(device)
+        self.copy_out = torch.cuda.Stream(device)
+        self.ev_in = [torch.cuda.Event() for _ in range(layers)]
+        self.ev_done = [torch.cuda.Event() for _ in range(layers)]
 
-    def call(self, li, s, prm, stream, e2e=False):
-        torch, B = self.torch, self.B
+    def call(self, li, s, prm, stream):
         lay = self.layers[li]
-        if e2e:
-            lay["q"][s].view(torch.int16).copy_(self.h_q[s], non_blocking=True)
-            lay["k_in"][s].view(torch.int16).copy_(self.h_k[s], non_blocking=True)
-            lay["v_in"][s].view(torch.int16).copy_(self.h_v[s], non_blocking=True)
-            lay["n"][s].copy_(self.h_n[s], non_blocking=True)
-        B.step(self.dp[s], prm, lay["cache"], lay["q"][s], lay["k_in"][s], lay["v_in"][s], lay["k_out"],
-               lay["v_out"], lay["n"][s], lay["a_full"], lay["ws"], l_full=lay["l_full"], decision_out=lay["dec"],
-               stream=stream)
-        if e2e:
-            tq = self.dp[s].host.total_q
-            self.h_a[li][:tq].copy_(lay["a_full"][:tq], non_blocking=True)
-            self.h_l[li][:tq].copy_(lay["l_full"][:tq], non_blocking=True)
+        self.B.step(self.dp[s], prm, lay["cache"], lay["q"][s], lay["k_in"][s], lay["v_in"][s], lay["k_out"],
+                    lay["v_out"], lay["n"][s], lay["a_full"], lay["ws"], l_full=lay["l_full"], decision_out=lay["dec"],
+                    stream=stream)
 
     def denoise_step(self, s, prm, stream, e2e=False):
         """Attention of every layer for denoise step s."""
+        if e2e:
+            return self.denoise_step_e2e(s, prm, stream)
         for li in range(self.L):
-            self.call(li, s, prm, stream, e2e)
+            self.call(li, s, prm, stream)
+
+    def denoise_step_e2e(self, s, prm, stream):
+        """The same with host buffers: each layer's block Q/K/V and update count are
+        uploaded from pinned memory and its A_full / L_full read back, the copies on
+        their own streams so that they overlap the other layers' attention."""
+        torch, B = self.torch, self.B
+        self.copy_in.wait_stream(stream)
+        self.copy_out.wait_stream(stream)
+        for li in range(self.L):
+            lay = self.layers[li]
+            with torch.cuda.stream(self.copy_in):
+                lay["inb"][s].copy_(self.h_in[s], non_blocking=True)  # Q, K_in, V_in, n_updated
+                self.ev_in[li].record(self.copy_in)
+            stream.wait_event(self.ev_in[li])
+            B.step(self.dp[s], prm, lay["cache"], lay["q"][s], lay["k_in"][s], lay["v_in"][s], lay["k_out"],
+                   lay["v_out"], lay["n"][s], lay["a_full"], lay["ws"], l_full=lay["l_full"], decision_out=lay["dec"],
+                   stream=stream)
+            self.ev_done[li].record(stream)
+            self.copy_out.wait_event(self.ev_done[li])
+            with torch.cuda.stream(self.copy_out):
+                self.h_out[li].copy_(lay["outb"], non_blocking=True)  # A_full, L_full
+        stream.wait_stream(self.copy_in)
+        stream.wait_stream(self.copy_out)
 
     def new_block(self, stream):
         """A new block starts: every layer's cache is empty (episode set-up, untimed)."""
@@ -299,11 +338,8 @@ class Model:
                 events[s][1].record(stream)
 
     def e2e_bytes(self, s):
-        st = self.w.steps[s]
-        tq = st.problem.total_q
-        H, d = self.w.problem.num_heads_q, self.w.problem.head_dim
-        return (st.q.nbytes + st.k_in.nbytes + st.v_in.nbytes + st.n_updated.astype(np.int32).nbytes,
-                tq * H * d * 2 + tq * H * 4)
+        """Bytes of the two copies of one call (the blobs, alignment padding included)."""
+        return int(self.h_in[s].numel()), int(self.out_bytes)
 
 
 def _events(torch, K, S):
