@@ -46,8 +46,9 @@ def _run(B, torch, w, use_noalloc):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("make", [lambda: W.dllm_layer(steps=2),
-                                  lambda: W.locking_tiny(steps=2)],
-                         ids=["dllm_layer", "locking_gqa"])
+                                  lambda: W.locking_tiny(steps=2),
+                                  lambda: W.video(steps=2, block=300, prefix_blocks=1, heads=4)],
+                         ids=["dllm_layer", "locking_gqa", "video_block_two_tile"])
 def test_noalloc_matches_fb_step(make):
     torch, B = torch_and_binding()
     w = make()
