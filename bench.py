@@ -490,7 +490,12 @@ def native(args, world, rank, local):
     reuse_b = step_bytes(p, 0.0)["total"]
     dense_med = float(np.median(dense_us))
     reuse_med = float(np.median(reuse_us))
-    n_launch = args.steps * S * L * (2 if w.flags & W.GATE_HEAD else 1)
+    # kernels per call: the attention kernel; the similarity kernel under the gamma
+    # gate; the work-order pass when the two-tile kernel runs with the gates on
+    gated = not (w.flags & (W.FORCE_RECOMPUTE | W.FORCE_REUSE))
+    two_tile = p.head_dim == 128 and p.num_heads_q == p.num_heads_kv and p.max_q >= 256
+    per_call = 1 + (1 if gated and w.flags & W.GATE_HEAD else 0) + (1 if gated and two_tile else 0)
+    n_launch = args.steps * S * L * per_call
     out = {
         "metric": METRIC,
         "value": round(value, 3),
