@@ -131,11 +131,11 @@ Shape shape_for(int d, int wm) {
       default: return shape_of<64, 8>();
     }
   }
+  // head_dim 128: groups of more than 64 rows (WM = 8) take the tensor-core kernel
   switch (wm) {
     case 1: return shape_of<128, 1>();
     case 2: return shape_of<128, 2>();
-    case 4: return shape_of<128, 4>();
-    default: return shape_of<128, 8>();
+    default: return shape_of<128, 4>();
   }
 }
 
