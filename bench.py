@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
                     [--workload dllm_layer|long_context_gqa|varlen_branches|video|tiny]
-                    [--layers L]
+                    [--layers L] [--rows]
 
 The workload is run the way a block-diffusion model runs it: every denoise step
 calls the attention of each of L layers (32 for the 8B dLLM), and every layer has
@@ -32,6 +32,11 @@ every launch.
 
 `--impl reference` times the fp64 oracle (the plain CPU statement of the method)
 on the host cores on one layer of the same workload, rank 0 only.
+
+`--rows` measures the extension rows instead (one JSON line, one GPU): the
+cumulative-M gate on the 8B-dLLM layer, the BlockBatch branch hooks on the
+varlen-branch problem, and the sparse-residual layout and step on the
+long-context GQA problem (see `rows`).
 
 With torchrun (N > 1) every rank runs its own request (seed + rank) on its own
 GPU with no collective on the data path (weak scaling); ranks meet only at the
@@ -104,6 +109,7 @@ class ClockSampler:
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
     def __init__(self, index: int, period_s: float = 0.005):
+        self.index = index
         self.samples = []
         self.max_mhz = None
         self.ok = False
@@ -555,6 +561,266 @@ def native(args, world, rank, local):
     _teardown(world)
 
 
+# ---------------------------------------------------------------- extension rows
+
+def sparse_selection(prefix_lens, seed: int = 7, sink: int = 64, window: int = 256, middle: int = 32):
+    """A static sparse pattern per sequence: the first `sink` prefix keys, the last
+    `window`, and `middle` seeded keys in between (increasing positions)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for n in prefix_lens:
+        n = int(n)
+        mid = rng.choice(np.arange(sink, n - window), size=middle, replace=False)
+        out.append(np.unique(np.concatenate([np.arange(sink), mid, np.arange(n - window, n)])).astype(np.int32))
+    return out
+
+
+def sparse_layout_bytes(p, total_sel: int) -> int:
+    """Bytes fb_sparse_layout must move: every prefix and block K/V row read once and
+    written once (to the residual prefix or the extended block), plus the indices."""
+    row = p.num_heads_kv * p.head_dim * 2 * 2          # K and V, bf16
+    return 2 * (p.total_kv_out + p.total_kv_in) * row + 4 * (total_sel + 3 * (p.num_seqs + 1))
+
+
+def cache_copy_bytes(p, src: int, dst: int, with_q_ref: bool) -> int:
+    """Bytes fb_cache_copy_seq must move: the entries of min(B_src, B_dst) block
+    positions (A_out fp32, L_out, and q_ref bf16 when the cache has it), read and
+    written, plus the per-head valid flags and update counts."""
+    n = min(int(p.lens("in")[src]), int(p.lens("in")[dst]))
+    per = p.num_heads_q * (p.head_dim * 4 + 4 + (p.head_dim * 2 if with_q_ref else 0))
+    return 2 * n * per + 2 * p.num_heads_q * 5
+
+
+def _graph_of(torch, fn):
+    """fn(stream) captured as a CUDA graph (run once eagerly first, outside capture)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn(side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    return g
+
+
+def _cold_us(torch, g, flush, flush_out, reps: int, clocks: "ClockSampler") -> np.ndarray:
+    """Device time of one replay of graph g, each after an untimed 256 MiB read that
+    evicts L2; CUDA events on the launching stream; µs per replay.  The SM clock
+    samples taken meanwhile are added to `clocks`."""
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    g.replay()
+    torch.cuda.synchronize()
+    with ClockSampler(clocks.index) as cs:
+        for e0, e1 in ev:
+            torch.amax(flush, dim=0, out=flush_out)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    clocks.samples += cs.samples
+    return np.array([e0.elapsed_time(e1) * 1e3 for e0, e1 in ev])
+
+
+def _stats(t: np.ndarray) -> dict:
+    return {"median": round(float(np.median(t)), 3), "p10": round(float(np.percentile(t, 10)), 3),
+            "p90": round(float(np.percentile(t, 90)), 3)}
+
+
+def _peaks() -> dict:
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        return {}
+
+
+class _Single:
+    """One layer of one step of a problem on the device: inputs, cache, workspace,
+    outputs (the shapes fb_step wants)."""
+
+    def __init__(self, B, torch, problem, st, k_out, v_out, device, with_q_ref=False):
+        self.B, self.dp = B, B.DeviceProblem(problem, device)
+        H, d = problem.num_heads_q, problem.head_dim
+        self.q = B.bf16_tensor(st.q, device)
+        self.k_in, self.v_in = B.bf16_tensor(st.k_in, device), B.bf16_tensor(st.v_in, device)
+        self.k_out, self.v_out = k_out, v_out
+        self.n = torch.as_tensor(st.n_updated.astype(np.int32)).to(device)
+        self.cache = B.Cache(problem, device, with_q_ref=with_q_ref)
+        self.ws = torch.empty(B.workspace_size(self.dp), dtype=torch.uint8, device=device)
+        B.workspace_init(self.ws)
+        self.a = torch.empty((max(problem.total_q, 1), H, d), dtype=torch.bfloat16, device=device)
+        self.l = torch.empty((max(problem.total_q, 1), H), dtype=torch.float32, device=device)
+
+    def step(self, prm, stream):
+        self.B.step(self.dp, prm, self.cache, self.q, self.k_in, self.v_in, self.k_out, self.v_out, self.n, self.a,
+                    self.ws, l_full=self.l, stream=stream)
+
+
+def rows(args, world, rank, local):
+    """Measurements of the extension rows on one GPU, one JSON line (rank 0 only):
+
+    * cumulative-M gate: the 8B-dLLM layer's episodes (L layers, graphs, L2 flushed
+      before every denoise step, as the headline) under FB_GATE_TAU_CUM, beside the
+      per-step gate on the same model;
+    * BlockBatch hooks on the varlen-branch problem: leader sync (fb_cache_copy_seq,
+      the 128-token branch's entries to the 64-token branch) and refresh
+      (fb_cache_invalidate_seqs of one branch), each after an L2 flush;
+    * sparse residual on the long-context GQA problem (8 x 32768 prefix): the layout
+      pass (fb_sparse_layout) and fb_step on the laid-out keys (forced recompute and
+      forced reuse), beside fb_step on the dense keys, each after an L2 flush."""
+    if rank != 0:
+        return
+    import dataclasses
+    import torch
+    from cached_split_attention_b200 import binding as B
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    flush = torch.ones(64 << 20, dtype=torch.int32, device=device)
+    flush_out = torch.empty((), dtype=torch.int32, device=device)
+    peaks = _peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
+    peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
+    reps = max(10, min(args.steps, 50))
+    out_rows, launches = {}, 0
+    clocks = ClockSampler(local)        # collects the samples of every timed region
+    # ---- cumulative-M gate (8B-dLLM layer)
+    w = make_workload("dllm_layer", 1001)
+    L = args.layers or DEFAULT_LAYERS["dllm_layer"]
+    model = Model(w, L, device)
+    S = model.S
+    stream = torch.cuda.current_stream()
+    lay0 = model.layers[0]
+    gate = {}
+    for name, flags in (("per_step", W.GATE_TAU), ("cumulative", W.GATE_TAU_CUM)):
+        prm = B.params(w.tau, w.gamma, flags)
+        B.cache_invalidate(model.dp[0], lay0["cache"], stream=stream)
+        rec = []
+        for s in range(S):
+            model.call(0, s, prm, stream)
+            rec.append(float(lay0["dec"].float().mean().item()))
+        for _ in range(args.warmup):
+            model.episode(flags)
+        ev = _events(torch, args.steps, S)
+        torch.cuda.synchronize()
+        with ClockSampler(local) as cs:
+            for k in range(args.steps):
+                model.episode(flags, events=ev[k])
+            torch.cuda.synchronize()
+        clocks.samples += cs.samples
+        launches += args.steps * S * L
+        step_us = _elapsed_us(ev)
+        rs = [s for s in range(S) if rec[s] > 0]
+        t_rec = step_us[:, rs].mean(axis=0) / L * 1e-6
+        b_rec = [step_bytes(w.steps[s].problem, rec[s])["total"] for s in rs]
+        ach = float(np.sum(b_rec) / np.sum(t_rec) / 1e9)
+        gate[name] = {"us_per_call": round(float(step_us.mean() / L), 3),
+                      "recompute_steps_per_episode": len(rs),
+                      "recompute_call_us": round(float(np.mean(t_rec)) * 1e6, 3),
+                      "roofline": {"bound": "hbm", "kernel": "attn_kernel, recompute launches",
+                                   "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                                   "frac": round(ach / hbm_peak, 4), "peak_source": peak_src}}
+    out_rows["cumulative_gate"] = dict(
+        workload=WORKLOAD_DESC["dllm_layer"] + f"; {L} layers, {S}-step episodes", tau=w.tau, **gate)
+    del model, lay0
+    torch.cuda.empty_cache()
+
+    # ---- BlockBatch hooks (varlen branches)
+    w = make_workload("varlen_branches", 1003)
+    p = w.problem
+    one = _Single(B, torch, p, w.steps[0], B.bf16_tensor(w.k_out, device), B.bf16_tensor(w.v_out, device),
+                  device)
+    one.step(B.params(0, 0.0, W.FORCE_RECOMPUTE), stream)   # fill every branch's entries
+    src, dst = int(np.argmax(p.lens("in"))), int(np.argsort(p.lens("in"))[-2])
+    mask = torch.zeros(p.num_seqs, dtype=torch.uint8, device=device)
+    mask[int(np.argmin(p.lens("in")))] = 1
+    g_copy = _graph_of(torch, lambda st: B.cache_copy_seq(one.dp, one.cache, src, dst, stream=st))
+    g_inv = _graph_of(torch, lambda st: B.cache_invalidate_seqs(one.dp, one.cache, mask, stream=st))
+    t_copy = _cold_us(torch, g_copy, flush, flush_out, reps, clocks)
+    t_inv = _cold_us(torch, g_inv, flush, flush_out, reps, clocks)
+    launches += 2 * reps
+    cb = cache_copy_bytes(p, src, dst, with_q_ref=False)
+    ach = cb / float(np.median(t_copy)) / 1e3
+    out_rows["branch_hooks"] = {
+        "workload": WORKLOAD_DESC["varlen_branches"],
+        "leader_sync": dict(_stats(t_copy), call="fb_cache_copy_seq", src_block=int(p.lens("in")[src]),
+                            dst_block=int(p.lens("in")[dst]), algorithmic_bytes=cb,
+                            roofline={"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak,
+                                      "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
+                                      "peak_source": peak_src}),
+        "refresh": dict(_stats(t_inv), call="fb_cache_invalidate_seqs", branches=1),
+    }
+    del one, g_copy, g_inv
+    torch.cuda.empty_cache()
+
+    # ---- sparse residual (long-context GQA)
+    w = make_workload("long_context_gqa", 1002)
+    p, st = w.problem, w.steps[0]
+    sel = sparse_selection(p.lens("out"))
+    cu_sel = np.concatenate([[0], np.cumsum([len(s) for s in sel])]).astype(np.int32)
+    total_sel = int(cu_sel[-1])
+    Hk, d = p.num_heads_kv, p.head_dim
+    k_out, v_out = B.bf16_tensor(w.k_out, device), B.bf16_tensor(w.v_out, device)
+    dense = _Single(B, torch, p, st, k_out, v_out, device)
+    k_res = torch.empty((p.total_kv_out - total_sel, Hk, d), dtype=torch.bfloat16, device=device)
+    v_res = torch.empty_like(k_res)
+    k_ext = torch.empty((p.total_kv_in + total_sel, Hk, d), dtype=torch.bfloat16, device=device)
+    v_ext = torch.empty_like(k_ext)
+    cu_o = torch.empty(p.num_seqs + 1, dtype=torch.int32, device=device)
+    cu_i = torch.empty(p.num_seqs + 1, dtype=torch.int32, device=device)
+    d_cu_sel = torch.as_tensor(cu_sel).to(device)
+    d_sel = torch.as_tensor(np.concatenate(sel)).to(device)
+
+    def layout(stream_):
+        B.sparse_layout(dense.dp, d_cu_sel, d_sel, total_sel, k_out, v_out, dense.k_in, dense.v_in, k_res, v_res,
+                        k_ext, v_ext, cu_o, cu_i, stream=stream_)
+
+    g_lay = _graph_of(torch, layout)
+    t_lay = _cold_us(torch, g_lay, flush, flush_out, reps, clocks)
+    p2 = dataclasses.replace(p, cu_seqlens_kv_out=cu_o.cpu().numpy(), cu_seqlens_kv_in=cu_i.cpu().numpy())
+    sp = _Single(B, torch, p2, dataclasses.replace(st, problem=p2), k_res, v_res, device)
+    sp.k_in, sp.v_in = k_ext, v_ext
+    timed = {}
+    for name, obj in (("sparse", sp), ("dense", dense)):
+        for arm, flags in (("recompute", W.FORCE_RECOMPUTE), ("reuse", W.FORCE_REUSE)):
+            prm = B.params(0, 0.0, flags)
+            g = _graph_of(torch, lambda st_, o=obj, pr=prm: o.step(pr, st_))
+            timed[(name, arm)] = _cold_us(torch, g, flush, flush_out, reps, clocks)
+            launches += reps
+            del g
+    launches += reps
+    if B.device_status() != 0:
+        raise RuntimeError("device status set during the sparse-residual measurement")
+    lb = sparse_layout_bytes(p, total_sel)
+    ach = lb / float(np.median(t_lay)) / 1e3
+
+    def arm(name, a, f):
+        t = timed[(name, a)]
+        b = step_bytes(p2 if name == "sparse" else p, f)["total"]
+        return dict(_stats(t), algorithmic_bytes=round(b), frac_of_hbm=round(b / float(np.median(t)) / 1e3 /
+                                                                             hbm_peak, 4))
+
+    out_rows["sparse_residual"] = {
+        "workload": WORKLOAD_DESC["long_context_gqa"],
+        "selection": f"per sequence the first 64 and last 256 prefix keys and 32 seeded keys between: "
+                     f"{total_sel // p.num_seqs} of {p.max_kv_out} keys",
+        "layout": dict(_stats(t_lay), call="fb_sparse_layout", algorithmic_bytes=lb,
+                       roofline={"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": round(ach / hbm_peak, 4), "peak_source": peak_src}),
+        "step_sparse": {"recompute_call_us": arm("sparse", "recompute", 1.0),
+                        "reuse_call_us": arm("sparse", "reuse", 0.0)},
+        "step_dense": {"recompute_call_us": arm("dense", "recompute", 1.0),
+                       "reuse_call_us": arm("dense", "reuse", 0.0)},
+    }
+    out = {"metric": "extension rows: device µs per call", "impl": "native", "bench": "rows", "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
+           "l2": "flushed (256 MiB read, untimed) before every timed denoise step or call",
+           "rows": out_rows, "gpu_launches": int(launches), "clocks": clocks.summary()}
+    print(json.dumps(out), flush=True)
+
+
 def _teardown(world):
     if world > 1:
         import torch.distributed as dist
@@ -642,11 +908,15 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=0, help="attention layers per denoise step (0: workload default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--rows", action="store_true",
+                    help="measure the extension rows (cumulative gate, branch hooks, sparse residual) instead")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
     world, rank, local = dist_setup()
-    if args.impl == "reference":
+    if args.rows and args.impl == "native":
+        rows(args, world, rank, local)
+    elif args.impl == "reference":
         reference(args, world, rank)
     else:
         native(args, world, rank, local)

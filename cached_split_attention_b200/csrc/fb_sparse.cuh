@@ -39,19 +39,19 @@ __global__ void __launch_bounds__(256) sparse_layout_kernel(const SparseParams p
   const int o0 = p.cu_out[b], n_out = p.cu_out[b + 1] - o0;
   const int i0 = p.cu_in[b], n_in = p.cu_in[b + 1] - i0;
   const int s0 = p.cu_sel[b], n_sel = p.cu_sel[b + 1] - s0;
-  __shared__ int s_ok;
-  if (threadIdx.x == 0) {
-    int ok = o0 >= 0 && n_out >= 0 && o0 + n_out <= p.total_out && i0 >= 0 && n_in >= 0 && i0 + n_in <= p.total_in &&
-             s0 >= 0 && n_sel >= 0 && s0 + n_sel <= p.total_sel && n_sel <= n_out;
-    for (int k = 0; ok && k < n_sel; ++k) {  // strictly increasing prefix positions
-      const int v = p.sel[s0 + k];
-      ok = v >= 0 && v < n_out && (k == 0 || v > p.sel[s0 + k - 1]);
-    }
-    if (!ok && blockIdx.x == 0) record_status(kDevBadIndex);
-    s_ok = ok;
+  // The whole CTA checks the ranges, then the selection (strictly increasing
+  // prefix positions), one element per thread per pass.
+  int ok = o0 >= 0 && n_out >= 0 && o0 + n_out <= p.total_out && i0 >= 0 && n_in >= 0 && i0 + n_in <= p.total_in &&
+           s0 >= 0 && n_sel >= 0 && s0 + n_sel <= p.total_sel && n_sel <= n_out;
+  for (int k = threadIdx.x; ok && k < n_sel; k += blockDim.x) {
+    const int v = p.sel[s0 + k];
+    ok = v >= 0 && v < n_out && (k == 0 || v > p.sel[s0 + k - 1]);
   }
-  __syncthreads();
-  if (!s_ok) return;
+  ok = __syncthreads_and(ok);
+  if (!ok) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_status(kDevBadIndex);
+    return;
+  }
   const int r0 = o0 - s0;  // J_out' of b starts here
   const int e0 = i0 + s0;  // J_in' of b starts here
   if (blockIdx.x == 0 && threadIdx.x == 0) {

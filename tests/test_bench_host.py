@@ -4,6 +4,7 @@ the maximum over ranks."""
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch.multiprocessing as mp
 
@@ -55,3 +56,25 @@ def test_step_bytes_dllm_layer():
     # Q 256 KiB + block K/V 512 KiB + A_full bf16 256 KiB + L 4 KiB + cache 516 KiB
     assert reuse == 262144 + 524288 + 266240 + 528384
     assert dense == reuse + 67108864
+
+
+def test_extension_row_byte_models():
+    """Byte models of the extension rows, counted by hand from the tensors."""
+    import bench
+    from cached_split_attention_b200 import workloads as W
+    p = W.varlen_branches(steps=1, prefix=64).problem
+    # 64 positions x 32 heads x (A_out 512 B + L_out 4 B), read and written, + valid and count
+    assert bench.cache_copy_bytes(p, 5, 4, with_q_ref=False) == 2 * 64 * 32 * 516 + 2 * 32 * 5
+    assert bench.cache_copy_bytes(p, 5, 4, with_q_ref=True) == 2 * 64 * 32 * 772 + 2 * 32 * 5
+    assert bench.cache_copy_bytes(p, 0, 5, with_q_ref=False) == 2 * 4 * 32 * 516 + 2 * 32 * 5
+    q = W.long_context_gqa(steps=1, batch=2, prefix=1000, heads_q=8, heads_kv=2).problem
+    # (2000 prefix + 128 block rows) x 2 heads x 128 x bf16 x (K, V), read and written, + indices
+    assert bench.sparse_layout_bytes(q, 10) == 2 * 2128 * 2 * 128 * 2 * 2 + 4 * (10 + 9)
+
+
+def test_sparse_selection_shape():
+    import bench
+    sel = bench.sparse_selection([32768, 1061])
+    for s, n in zip(sel, [32768, 1061]):
+        assert len(s) == 64 + 32 + 256 and np.all(np.diff(s) > 0) and s[0] == 0 and s[-1] == n - 1
+        assert np.array_equal(s[:64], np.arange(64)) and np.array_equal(s[-256:], np.arange(n - 256, n))
