@@ -673,7 +673,6 @@ def rows(args, world, rank, local):
       forced reuse), beside fb_step on the dense keys, each after an L2 flush."""
     if rank != 0:
         return
-    import dataclasses
     import torch
     from cached_split_attention_b200 import binding as B
     torch.cuda.set_device(local)
@@ -686,7 +685,26 @@ def rows(args, world, rank, local):
     reps = max(10, min(args.steps, 50))
     out_rows, launches = {}, 0
     clocks = ClockSampler(local)        # collects the samples of every timed region
-    # ---- cumulative-M gate (8B-dLLM layer)
+    stream = torch.cuda.current_stream()
+    if args.rows in ("all", "gate"):
+        launches += _rows_gate(args, torch, B, device, local, clocks, out_rows, hbm_peak, peak_src)
+    if args.rows in ("all", "hooks"):
+        launches += _rows_hooks(torch, B, device, stream, flush, flush_out, reps, clocks, out_rows, hbm_peak,
+                                peak_src)
+    if args.rows in ("all", "sparse"):
+        launches += _rows_sparse(torch, B, device, flush, flush_out, reps, clocks, out_rows, hbm_peak, peak_src)
+    if B.device_status() != 0:
+        raise RuntimeError("device status set during the extension-row measurements")
+    out = {"metric": "extension rows: device µs per call", "impl": "native", "bench": "rows", "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
+           "l2": "flushed (256 MiB read, untimed) before every timed denoise step or call",
+           "rows": out_rows, "gpu_launches": int(launches), "clocks": clocks.summary()}
+    print(json.dumps(out), flush=True)
+
+
+def _rows_gate(args, torch, B, device, local, clocks, out_rows, hbm_peak, peak_src) -> int:
+    """Cumulative-M gate against the per-step gate, 8B-dLLM layer episodes."""
+    launches = 0
     w = make_workload("dllm_layer", 1001)
     L = args.layers or DEFAULT_LAYERS["dllm_layer"]
     model = Model(w, L, device)
@@ -726,8 +744,13 @@ def rows(args, world, rank, local):
         workload=WORKLOAD_DESC["dllm_layer"] + f"; {L} layers, {S}-step episodes", tau=w.tau, **gate)
     del model, lay0
     torch.cuda.empty_cache()
+    return launches
 
-    # ---- BlockBatch hooks (varlen branches)
+
+def _rows_hooks(torch, B, device, stream, flush, flush_out, reps, clocks, out_rows, hbm_peak, peak_src) -> int:
+    """BlockBatch leader sync and refresh on the varlen-branch problem: one call
+    after an L2 flush, and 32 calls back to back in one graph (per-call time)."""
+    launches = 0
     w = make_workload("varlen_branches", 1003)
     p = w.problem
     one = _Single(B, torch, p, w.steps[0], B.bf16_tensor(w.k_out, device), B.bf16_tensor(w.v_out, device),
@@ -736,11 +759,15 @@ def rows(args, world, rank, local):
     src, dst = int(np.argmax(p.lens("in"))), int(np.argsort(p.lens("in"))[-2])
     mask = torch.zeros(p.num_seqs, dtype=torch.uint8, device=device)
     mask[int(np.argmin(p.lens("in")))] = 1
-    g_copy = _graph_of(torch, lambda st: B.cache_copy_seq(one.dp, one.cache, src, dst, stream=st))
-    g_inv = _graph_of(torch, lambda st: B.cache_invalidate_seqs(one.dp, one.cache, mask, stream=st))
-    t_copy = _cold_us(torch, g_copy, flush, flush_out, reps, clocks)
-    t_inv = _cold_us(torch, g_inv, flush, flush_out, reps, clocks)
-    launches += 2 * reps
+    copy = lambda st: B.cache_copy_seq(one.dp, one.cache, src, dst, stream=st)
+    inv = lambda st: B.cache_invalidate_seqs(one.dp, one.cache, mask, stream=st)
+    t_copy = _cold_us(torch, _graph_of(torch, copy), flush, flush_out, reps, clocks)
+    t_inv = _cold_us(torch, _graph_of(torch, inv), flush, flush_out, reps, clocks)
+    nb = 32
+    many = lambda fn: (lambda st: [fn(st) for _ in range(nb)])
+    t_copy_bb = _cold_us(torch, _graph_of(torch, many(copy)), flush, flush_out, reps, clocks) / nb
+    t_inv_bb = _cold_us(torch, _graph_of(torch, many(inv)), flush, flush_out, reps, clocks) / nb
+    launches += 2 * reps * (1 + nb)
     cb = cache_copy_bytes(p, src, dst, with_q_ref=False)
     ach = cb / float(np.median(t_copy)) / 1e3
     out_rows["branch_hooks"] = {
@@ -749,13 +776,23 @@ def rows(args, world, rank, local):
                             dst_block=int(p.lens("in")[dst]), algorithmic_bytes=cb,
                             roofline={"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak,
                                       "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
-                                      "peak_source": peak_src}),
-        "refresh": dict(_stats(t_inv), call="fb_cache_invalidate_seqs", branches=1),
+                                      "peak_source": peak_src},
+                            back_to_back_us_per_call=_stats(t_copy_bb)),
+        "refresh": dict(_stats(t_inv), call="fb_cache_invalidate_seqs", branches=1,
+                        back_to_back_us_per_call=_stats(t_inv_bb)),
+        "timing": f"median over {reps} graph replays, each after an L2 flush; back to back: "
+                  f"{nb} calls in one graph, time / {nb}",
     }
-    del one, g_copy, g_inv
+    del one
     torch.cuda.empty_cache()
+    return launches
 
-    # ---- sparse residual (long-context GQA)
+
+def _rows_sparse(torch, B, device, flush, flush_out, reps, clocks, out_rows, hbm_peak, peak_src) -> int:
+    """Sparse residual on the long-context GQA problem: the layout pass, and fb_step
+    on the laid-out keys beside fb_step on the dense keys (forced recompute / reuse)."""
+    import dataclasses
+    launches = 0
     w = make_workload("long_context_gqa", 1002)
     p, st = w.problem, w.steps[0]
     sel = sparse_selection(p.lens("out"))
@@ -791,8 +828,6 @@ def rows(args, world, rank, local):
             launches += reps
             del g
     launches += reps
-    if B.device_status() != 0:
-        raise RuntimeError("device status set during the sparse-residual measurement")
     lb = sparse_layout_bytes(p, total_sel)
     ach = lb / float(np.median(t_lay)) / 1e3
 
@@ -814,11 +849,7 @@ def rows(args, world, rank, local):
         "step_dense": {"recompute_call_us": arm("dense", "recompute", 1.0),
                        "reuse_call_us": arm("dense", "reuse", 0.0)},
     }
-    out = {"metric": "extension rows: device µs per call", "impl": "native", "bench": "rows", "n_gpus": 1,
-           "steps": args.steps, "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
-           "l2": "flushed (256 MiB read, untimed) before every timed denoise step or call",
-           "rows": out_rows, "gpu_launches": int(launches), "clocks": clocks.summary()}
-    print(json.dumps(out), flush=True)
+    return launches
 
 
 def _teardown(world):
@@ -908,7 +939,7 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=0, help="attention layers per denoise step (0: workload default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
-    ap.add_argument("--rows", action="store_true",
+    ap.add_argument("--rows", nargs="?", const="all", default=None, choices=["all", "gate", "hooks", "sparse"],
                     help="measure the extension rows (cumulative gate, branch hooks, sparse residual) instead")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "native":
