@@ -21,6 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libflashblock.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 GATE_TAU, GATE_HEAD, FORCE_RECOMPUTE, FORCE_REUSE, GATE_TAU_CUM = 1, 2, 4, 8, 16
+CALL_STEP, CALL_OUT, CALL_IN = 0, 1, 2
+KERNEL_NAMES = {0: "attn_kernel", 1: "tc_attn_kernel", 2: "tc2_attn_kernel"}
 
 
 class FlashBlockError(RuntimeError):
@@ -51,6 +53,11 @@ class FbParams(ctypes.Structure):
     _fields_ = [("tau", ctypes.c_int32), ("gamma", ctypes.c_float), ("flags", ctypes.c_uint32)]
 
 
+class FbPlanInfo(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("kernel", "rows_per_tile", "tiles", "work_items", "splits", "ctas",
+                                              "threads", "smem_bytes", "keys_per_chunk", "num_sms")]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python -m cached_split_attention_b200.build`")
@@ -61,6 +68,7 @@ def _load():
         "fb_last_error": (ctypes.c_char_p, []),
         "fb_version": (ctypes.c_int32, []),
         "fb_workspace_size": (st, [P, ctypes.POINTER(sz)]),
+        "fb_plan_query": (st, [P, ctypes.c_int32, ctypes.POINTER(FbPlanInfo)]),
         "fb_workspace_init": (st, [vp, sz, vp]),
         "fb_out_attn": (st, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "fb_in_attn": (st, [P, vp, vp, vp, vp, vp, vp]),
@@ -166,6 +174,16 @@ def params(tau: int = 0, gamma: float = 0.0, flags: int = 0) -> FbParams:
 
 
 # ---------------------------------------------------------------- calls
+
+def plan_query(problem: DeviceProblem, call: int = CALL_STEP) -> dict:
+    """fb_plan_query: the launch plan of a call as a dict (plus ``kernel_name``).
+    Host computation only; the problem's index arrays may live on the host."""
+    info = FbPlanInfo()
+    _check(_lib.fb_plan_query(problem.ref, int(call), ctypes.byref(info)))
+    out = {name: int(getattr(info, name)) for name, _ in FbPlanInfo._fields_}
+    out["kernel_name"] = KERNEL_NAMES[out["kernel"]]
+    return out
+
 
 def workspace_size(problem: DeviceProblem) -> int:
     n = ctypes.c_size_t(0)

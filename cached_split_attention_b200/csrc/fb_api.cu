@@ -350,6 +350,27 @@ const char* fb_last_error(void) { return t_err.c_str(); }
 
 int32_t fb_version(void) { return 100; }
 
+fb_status fb_plan_query(const fb_problem* problem, int32_t call, fb_plan_info* out) {
+  FB_TRY(check_problem(problem));
+  if (!out) return fail(FB_ERR_INVALID_ARG, "out is NULL");
+  if (call != FB_CALL_STEP && call != FB_CALL_OUT && call != FB_CALL_IN)
+    return fail(FB_ERR_INVALID_ARG, "unknown call %d", call);
+  const int sms = device_sms();
+  const Plan pl = make_plan(problem, sms, call == FB_CALL_IN, call == FB_CALL_STEP);
+  out->kernel = pl.tc2 ? FB_KERNEL_TC2 : pl.tc ? FB_KERNEL_TC : FB_KERNEL_WARP_MMA;
+  out->rows_per_tile = pl.tc2 ? pl.tr / 2 : pl.tr;
+  const long rows = static_cast<long>(pl.g) * problem->max_q;
+  out->tiles = pl.tc2 ? static_cast<int>(std::max<long>(1, (rows + pl.tr / 2 - 1) / (pl.tr / 2))) : pl.tiles;
+  out->work_items = pl.n_groups;
+  out->splits = pl.splits;
+  out->ctas = pl.n_groups * pl.splits;
+  out->threads = pl.threads;
+  out->smem_bytes = pl.smem;
+  out->keys_per_chunk = pl.bn;
+  out->num_sms = sms;
+  return FB_OK;
+}
+
 fb_status fb_workspace_size(const fb_problem* problem, size_t* bytes) {
   FB_TRY(check_problem(problem));
   if (!bytes) return fail(FB_ERR_INVALID_ARG, "bytes is NULL");

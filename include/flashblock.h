@@ -128,6 +128,44 @@ const char* fb_last_error(void);
 /* Library version (major*100 + minor). */
 int32_t fb_version(void);
 
+/* Calls whose launch plan fb_plan_query describes. */
+#define FB_CALL_STEP 0 /* fb_step (and fb_step_noalloc)  */
+#define FB_CALL_OUT 1  /* fb_out_attn                     */
+#define FB_CALL_IN 2   /* fb_in_attn                      */
+
+/* Attention kernels a plan may choose. */
+#define FB_KERNEL_WARP_MMA 0 /* attn_kernel: warp-level MMA, groups of up to 64 rows (all head_dim 64)  */
+#define FB_KERNEL_TC 1       /* tc_attn_kernel: tcgen05 with TMEM accumulators, one 128-row tile       */
+#define FB_KERNEL_TC2 2      /* tc2_attn_kernel: tcgen05, two 128-row tiles of one head per CTA       */
+
+/*
+ * Launch plan of the attention kernel of one call.  A group is the rows of one
+ * (sequence, kv-head): its block rows times the query heads sharing the kv-head,
+ * cut into tiles of rows_per_tile.  Each tile's prefix keys are split over
+ * `splits` CTAs of one cluster, whose partials are combined in distributed shared
+ * memory (splits = 1: no cluster).
+ */
+typedef struct fb_plan_info {
+  int32_t kernel;         /* FB_KERNEL_*                                          */
+  int32_t rows_per_tile;  /* query rows (token x q-head of the group) per tile     */
+  int32_t tiles;          /* tiles per group                                       */
+  int32_t work_items;     /* (sequence, kv-head, tile) items (two-tile kernel: pairs) */
+  int32_t splits;         /* CTAs per item over the prefix keys (cluster size)      */
+  int32_t ctas;           /* grid size = work_items x splits                        */
+  int32_t threads;        /* threads per CTA                                        */
+  int32_t smem_bytes;     /* dynamic shared memory per CTA                          */
+  int32_t keys_per_chunk; /* keys per pipeline stage (TMA box rows)                 */
+  int32_t num_sms;        /* SM count the plan was made for                         */
+} fb_plan_info;
+
+/*
+ * The launch plan `call` (FB_CALL_*) would use for this problem on the current
+ * device (148 SMs when no device is visible).  Pure host computation: the
+ * cu_seqlens pointers are not read.  FB_ERR_INVALID_ARG for a bad problem, an
+ * unknown call or a NULL out.
+ */
+fb_status fb_plan_query(const fb_problem* problem, int32_t call, fb_plan_info* out);
+
 /*
  * Bytes of workspace that fb_out_attn / fb_step need for this problem (a
  * completion counter and the per-head similarity scores; partials stay on chip).

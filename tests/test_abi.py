@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -118,3 +119,61 @@ def test_workspace_size_is_counter_plus_scores():
                     max_kv_in=1560)
     assert B._lib.fb_workspace_size(ctypes.byref(prob), ctypes.byref(n)) == B.OK
     assert n.value == 256 + 256 + 1280, n.value  # 40 x 7 items x 4 bytes = 1120 -> 1280
+
+
+def _shape_problems():
+    """The step-0 problems of the bench workloads (shapes only; no K/V drawn)."""
+    from cached_split_attention_b200.workloads import make_problem
+    rng = np.random.default_rng(0)
+    return {
+        "dllm_layer": make_problem([np.arange(32)], [4096], [32], 32, 32, 128),
+        "tiny": make_problem([np.arange(32)], [256], [32], 4, 4, 64),
+        "long_context_gqa": make_problem([np.sort(rng.permutation(64)[:32]) for _ in range(8)], [32768] * 8,
+                                         [64] * 8, 32, 8, 128),
+        "varlen_branches": make_problem([np.arange(b) for b in (4, 8, 16, 32, 64, 128)], [2048] * 6,
+                                        [4, 8, 16, 32, 64, 128], 32, 32, 128),
+        "video": make_problem([np.arange(1560)], [9360], [1560], 40, 40, 128),
+    }
+
+
+def test_plan_query_matches_the_bench_kernel_map():
+    """fb_plan_query on the CPU: the fused step of each bench workload takes the
+    kernel bench.py attributes its roofline and counters to; the grid is items x
+    splits; the two-tile kernel and the block-only pass never split the prefix; the
+    warp-MMA kernel's split grid fits one wave."""
+    _built()
+    import bench
+    from cached_split_attention_b200 import binding as B
+    for name, p in _shape_problems().items():
+        dp = B.DeviceProblem(p, "cpu")
+        step = B.plan_query(dp, B.CALL_STEP)
+        assert step["kernel_name"] == bench.KERNEL_OF[name], (name, step)
+        for call in (B.CALL_STEP, B.CALL_OUT, B.CALL_IN):
+            pl = B.plan_query(dp, call)
+            assert pl["ctas"] == pl["work_items"] * pl["splits"] > 0, (name, call, pl)
+            assert 1 <= pl["splits"] <= 16
+            if call == B.CALL_IN or pl["kernel"] == 2:
+                assert pl["splits"] == 1, (name, call, pl)
+            if pl["kernel"] == 0 and call != B.CALL_IN and pl["splits"] > 1:
+                per_sm = max(1, min(233472 // (pl["smem_bytes"] + 1024), 2048 // pl["threads"]))
+                assert pl["ctas"] <= pl["num_sms"] * per_sm, (name, pl)
+        # the unfused prefix pass never takes the two-tile kernel (that is fb_step's)
+        assert B.plan_query(dp, B.CALL_OUT)["kernel"] != 2
+    video = B.plan_query(B.DeviceProblem(_shape_problems()["video"], "cpu"))
+    assert (video["rows_per_tile"], video["tiles"], video["work_items"]) == (128, 13, 40 * 7)
+    dllm = B.plan_query(B.DeviceProblem(_shape_problems()["dllm_layer"], "cpu"))
+    assert (dllm["rows_per_tile"], dllm["tiles"], dllm["work_items"]) == (32, 1, 32)
+    gqa = B.plan_query(B.DeviceProblem(_shape_problems()["long_context_gqa"], "cpu"))
+    assert (gqa["rows_per_tile"], gqa["tiles"], gqa["work_items"]) == (128, 1, 64)
+
+
+def test_plan_query_rejects_bad_arguments():
+    _built()
+    from cached_split_attention_b200 import binding as B
+    ok = _problem(B)
+    info = B.FbPlanInfo()
+    assert B._lib.fb_plan_query(ctypes.byref(ok), 3, ctypes.byref(info)) == B.ERR_INVALID_ARG
+    assert "unknown call" in B.last_error()
+    assert B._lib.fb_plan_query(ctypes.byref(ok), 0, None) == B.ERR_INVALID_ARG
+    bad = _problem(B, head_dim=96)
+    assert B._lib.fb_plan_query(ctypes.byref(bad), 0, ctypes.byref(info)) == B.ERR_UNSUPPORTED
