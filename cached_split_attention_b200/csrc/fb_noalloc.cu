@@ -16,8 +16,10 @@
 
 namespace {
 
-// Largest scratch a call may need: a 256-byte completion-counter slot plus one
-// fp32 similarity score per (sequence, q-head), i.e. up to 16320 such pairs.
+// Scratch of every call: a call runs when its fb_workspace_size fits here -- a
+// 256-byte completion-counter slot plus one fp32 similarity score per (sequence,
+// q-head), i.e. up to 16320 such pairs, fewer when the workspace also holds the
+// two-tile kernel's work order (one int32 per (sequence, head, 256-row pair)).
 constexpr size_t kScratchBytes = 64 * 1024;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];

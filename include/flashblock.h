@@ -319,8 +319,10 @@ fb_status fb_device_status(int32_t* code, fb_stream_t stream);
  *
  * Arguments and results are those of fb_step.  Instead of a caller workspace the
  * call uses a scratch array built into the library: 64 KiB of device memory that
- * every GPU loading the library holds until the process exits.  It covers
- * num_seqs x num_heads_q up to 16320; larger problems return FB_ERR_UNSUPPORTED
+ * every GPU loading the library holds until the process exits.  It covers every
+ * problem whose fb_workspace_size is at most 64 KiB: num_seqs x num_heads_q up to
+ * 16320, fewer for multi-head problems of 256+ rows per head (their workspace also
+ * holds the two-tile work order).  Larger problems return FB_ERR_UNSUPPORTED
  * (message in fb_noalloc_last_error()) -- use fb_step with a workspace for them.
  * No call allocates: the first call on a device resolves the scratch address
  * (cudaGetSymbolAddress), so make that first call before capturing a stream.
