@@ -869,6 +869,20 @@ def _oracle_threads():
         return os.cpu_count() or 1
 
 
+def host_cpu() -> dict:
+    """The host the oracle runs on: logical CPUs (nproc) and the CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_baseline(workload: str, seed: int, budget_s: float = 12.0) -> dict:
     """The fp64 oracle (as it stands) on a bounded sample: whole episodes of the
     same workload until about budget_s seconds have passed."""
@@ -884,7 +898,7 @@ def cpu_baseline(workload: str, seed: int, budget_s: float = 12.0) -> dict:
             break
     dt = time.perf_counter() - t0
     return {"value": round(dt / (n * S) * 1e6, 1), "unit": "us/attention-call (one layer, one denoise step)",
-            "cores": _oracle_threads(), "kind": "oracle",
+            "cores": _oracle_threads(), "host": host_cpu(), "kind": "oracle",
             "sample": f"{n} full episode(s) of {S} denoise steps of one layer, every row and head, fp64 numpy"}
 
 
@@ -921,7 +935,7 @@ def reference(args, world, rank):
         "config": {"workload": WORKLOAD_DESC[args.workload],
                    "bench_step": f"one denoise episode ({S} steps) of one layer, fp64 oracle on host cores"},
         "cpu_baseline": {"value": round(us, 1), "unit": "us/attention-call (one layer, one denoise step)",
-                         "cores": cores, "kind": "oracle",
+                         "cores": cores, "host": host_cpu(), "kind": "oracle",
                          "sample": f"{args.steps} full episode(s) of {S} denoise steps of one layer, every row and head"},
         "e2e": {"value": round(us, 1), "unit": "us/attention-call (one layer, one denoise step)",
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -78,3 +78,12 @@ def test_sparse_selection_shape():
     for s, n in zip(sel, [32768, 1061]):
         assert len(s) == 64 + 32 + 256 and np.all(np.diff(s) > 0) and s[0] == 0 and s[-1] == n - 1
         assert np.array_equal(s[:64], np.arange(64)) and np.array_equal(s[-256:], np.arange(n - 256, n))
+
+
+def test_cpu_baseline_reports_its_host():
+    """The oracle baseline states the threads it used, nproc and the CPU model."""
+    import bench
+    out = bench.cpu_baseline("tiny", 1000, budget_s=0.05)
+    assert out["kind"] == "oracle" and out["value"] > 0 and out["cores"] >= 1
+    assert out["host"]["nproc"] == os.cpu_count()
+    assert out["host"]["cpu_model"] is None or isinstance(out["host"]["cpu_model"], str)
