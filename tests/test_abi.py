@@ -177,3 +177,54 @@ def test_plan_query_rejects_bad_arguments():
     assert B._lib.fb_plan_query(ctypes.byref(ok), 0, None) == B.ERR_INVALID_ARG
     bad = _problem(B, head_dim=96)
     assert B._lib.fb_plan_query(ctypes.byref(bad), 0, ctypes.byref(info)) == B.ERR_UNSUPPORTED
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "flashblock.h"
+
+int main(void) {
+  /* 1 sequence, MHA 32 heads, d 128, prefix 4096, block 32 (host-only calls: the
+     index arrays are not read, so host arrays serve) */
+  static const int32_t cu_q[2] = {0, 32}, cu_out[2] = {0, 4096}, cu_in[2] = {0, 32};
+  fb_problem p;
+  memset(&p, 0, sizeof(p));
+  p.num_seqs = 1; p.num_heads_q = 32; p.num_heads_kv = 32; p.head_dim = 128;
+  p.softmax_scale = 0.08838834764831845f;
+  p.cu_seqlens_q = cu_q; p.cu_seqlens_kv_out = cu_out; p.cu_seqlens_kv_in = cu_in;
+  p.total_q = 32; p.total_kv_out = 4096; p.total_kv_in = 32;
+  p.max_q = 32; p.max_kv_out = 4096; p.max_kv_in = 32;
+  size_t ws = 0;
+  if (fb_workspace_size(&p, &ws) != FB_OK) return 2;
+  fb_plan_info info;
+  if (fb_plan_query(&p, FB_CALL_STEP, &info) != FB_OK) return 3;
+  p.head_dim = 96;
+  if (fb_workspace_size(&p, &ws) != FB_ERR_UNSUPPORTED || strlen(fb_last_error()) == 0) return 4;
+  printf("%d %zu %d %d %d\n", fb_version(), ws, info.kernel, info.work_items, info.ctas);
+  return 0;
+}
+"""
+
+
+def test_header_serves_a_plain_c_caller(tmp_path):
+    """The boundary is C: a C99 program includes flashblock.h, links the library and
+    makes host-only calls (no GPU needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib = _built()
+    src = tmp_path / "caller.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(lib)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-L", libdir, "-lflashblock", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    version, ws, kernel, items, ctas = map(int, r.stdout.split())
+    assert version >= 100 and ws == 512 and kernel == 0 and items == 32 and ctas == 128
