@@ -62,6 +62,12 @@ fb_status check_problem(const fb_problem* p) {
   if (static_cast<int64_t>(p->total_kv_in) * p->num_heads_q >= (int64_t{1} << 31) ||
       static_cast<int64_t>(p->total_q) * p->num_heads_q >= (int64_t{1} << 31))
     return fail(FB_ERR_UNSUPPORTED, "tokens x query heads must stay below 2^31");
+  // The grid has up to num_seqs x num_heads_q x max_q x kMaxSplits CTAs (every
+  // sequence is sized by the longest); keep it, and the per-(sequence, head)
+  // workspace arrays, inside 32-bit indices.
+  if (static_cast<int64_t>(p->num_seqs) * p->num_heads_q * std::max(1, p->max_q) * fb::kMaxSplits >=
+      (int64_t{1} << 31))
+    return fail(FB_ERR_UNSUPPORTED, "num_seqs x num_heads_q x max_q is too large for one launch");
   if (p->num_seqs > 0 && (!p->cu_seqlens_q || !p->cu_seqlens_kv_out || !p->cu_seqlens_kv_in))
     return fail(FB_ERR_INVALID_ARG, "cu_seqlens arrays must not be NULL");
   return FB_OK;

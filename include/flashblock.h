@@ -55,7 +55,8 @@ typedef struct CUstream_st* fb_stream_t; /* same type as cudaStream_t; NULL = de
 typedef enum fb_status {
   FB_OK = 0,
   FB_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned buffer, bad offsets */
-  FB_ERR_UNSUPPORTED = 2, /* head_dim not 64/128, num_heads_q % num_heads_kv != 0, group > 32 */
+  FB_ERR_UNSUPPORTED = 2, /* head_dim not 64/128, num_heads_q % num_heads_kv != 0, group > 32,
+                             sizes past 32-bit launch indices */
   FB_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed (message has the CUDA error) */
   FB_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out (see fb_device_status) */
 } fb_status;

@@ -228,3 +228,39 @@ def test_header_serves_a_plain_c_caller(tmp_path):
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     version, ws, kernel, items, ctas = map(int, r.stdout.split())
     assert version >= 100 and ws == 512 and kernel == 0 and items == 32 and ctas == 128
+
+
+def test_host_checks_hold_for_any_problem_fields():
+    """Random (also absurd) fb_problem fields: the host-only calls answer OK or an
+    argument/unsupported error, never crash; an accepted problem's workspace holds
+    the counter slot and one fp32 score per (sequence, q-head), and its plan's grid
+    is work items x splits."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+    _built()
+    from cached_split_attention_b200 import binding as B
+    i32 = st.one_of(st.integers(-3, 70), st.integers(0, 1 << 20),
+                    st.sampled_from([2 ** 31 - 1, -2 ** 31, 2 ** 30, 600_000_000, 1 << 16]))
+
+    @settings(max_examples=400, deadline=None)
+    @given(ns=i32, hq=i32, hkv=st.sampled_from([1, 2, 4, 8, 0, -1]), d=st.sampled_from([64, 128, 96]), tq=i32,
+           to=i32, ti=i32, mq=i32, mo=i32, mi=i32, sp=st.integers(-1, 20), call=st.integers(-1, 3))
+    def check(ns, hq, hkv, d, tq, to, ti, mq, mo, mi, sp, call):
+        p = B.FbProblem(ns, hq, hkv, d, 0.1, 16, 0, 16, 16, tq, to, ti, mq, mo, mi, sp)
+        n = ctypes.c_size_t()
+        rc = B._lib.fb_workspace_size(ctypes.byref(p), ctypes.byref(n))
+        assert rc in (B.OK, B.ERR_INVALID_ARG, B.ERR_UNSUPPORTED)
+        if rc == B.OK:
+            assert n.value >= 256 + 4 * ns * hq, (ns, hq, n.value)
+        info = B.FbPlanInfo()
+        rc = B._lib.fb_plan_query(ctypes.byref(p), call, ctypes.byref(info))
+        assert rc in (B.OK, B.ERR_INVALID_ARG, B.ERR_UNSUPPORTED)
+        if rc == B.OK:
+            assert info.ctas == info.work_items * info.splits >= 0 and 1 <= info.splits <= 16
+
+    check()
+    # the overflow this guards against: 600M sequences x 4 heads
+    big = _problem(B, num_seqs=600_000_000, num_heads_q=4, num_heads_kv=4, total_q=0, max_q=0, total_kv_in=0,
+                   max_kv_in=0, total_kv_out=0, max_kv_out=0)
+    n = ctypes.c_size_t()
+    assert B._lib.fb_workspace_size(ctypes.byref(big), ctypes.byref(n)) == B.ERR_UNSUPPORTED
