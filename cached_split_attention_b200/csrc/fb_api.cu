@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -446,6 +447,7 @@ fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16*
 fb_status fb_merge(int64_t n, int32_t d, const float* a_out, const float* l_out, const float* a_in,
                    const float* l_in, float* a_full_f32, fb_bf16* a_full_bf16, float* l_full, fb_stream_t stream) {
   if (n < 0 || d <= 0) return fail(FB_ERR_INVALID_ARG, "n must be >= 0 and d > 0");
+  if (n > INT64_MAX / d) return fail(FB_ERR_INVALID_ARG, "n x d overflows 64 bits");
   if (n == 0) return FB_OK;
   if (!a_out || !l_out || !a_in || !l_in) return fail(FB_ERR_INVALID_ARG, "merge inputs must not be NULL");
   if (!a_full_f32 && !a_full_bf16) return fail(FB_ERR_INVALID_ARG, "no output for A_full");

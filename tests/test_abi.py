@@ -91,6 +91,8 @@ def test_host_validation_without_gpu():
                         16, 16, None, 16, 1 << 30, None)
     assert rc == B.ERR_INVALID_ARG and "unknown flag" in B.last_error()
     assert B._lib.fb_merge(-1, 4, 16, 16, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG
+    assert B._lib.fb_merge(2 ** 62, 4, 16, 16, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG
+    assert "overflows" in B.last_error()
     # branch hooks and the sparse layout: argument checks before any device work
     cache5 = B.FbCache(16, 16, 16, 0, 0)
     assert B._lib.fb_cache_copy_seq(ctypes.byref(ok), ctypes.byref(cache5), 0, 3, None) == B.ERR_INVALID_ARG
