@@ -612,6 +612,8 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
   if (total_sel < 0 || total_sel > problem->total_kv_out)
     return fail(FB_ERR_INVALID_ARG, "total_sel %d outside [0, total_kv_out]", total_sel);
   if (problem->num_seqs == 0) return FB_OK;
+  if (problem->num_seqs > 65535)  // one grid row per sequence
+    return fail(FB_ERR_UNSUPPORTED, "fb_sparse_layout takes at most 65535 sequences per call");
   if (!cu_sel) return fail(FB_ERR_INVALID_ARG, "cu_sel is NULL");
   if (total_sel > 0 && !sel_idx) return fail(FB_ERR_INVALID_ARG, "sel_idx is NULL");
   const bool res = problem->total_kv_out - total_sel > 0;

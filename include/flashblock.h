@@ -286,7 +286,7 @@ fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* ca
  * full attention over prefix and block.  The selection is fixed for a block (a new one
  * changes the residual: refill the cache).  A selection that is not increasing or out of
  * range records FB_ERR_INVALID_ARG on the device (fb_device_status); that sequence is
- * skipped.
+ * skipped.  At most 65535 sequences per call (FB_ERR_UNSUPPORTED beyond).
  */
 fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, const int32_t* sel_idx,
                            int32_t total_sel, const fb_bf16* k_out, const fb_bf16* v_out, const fb_bf16* k_in,

@@ -102,6 +102,9 @@ def test_host_validation_without_gpu():
     assert rc == B.ERR_INVALID_ARG and "total_sel" in B.last_error()
     rc = B._lib.fb_sparse_layout(ctypes.byref(ok), None, 16, 4, 16, 16, 16, 16, 16, 16, 16, 16, None, None, None)
     assert rc == B.ERR_INVALID_ARG and "cu_sel" in B.last_error()
+    many = _problem(B, num_seqs=70000, total_q=0, max_q=0, total_kv_in=0, max_kv_in=0, total_kv_out=0, max_kv_out=0)
+    rc = B._lib.fb_sparse_layout(ctypes.byref(many), 16, 16, 0, 16, 16, 16, 16, 16, 16, 16, 16, None, None, None)
+    assert rc == B.ERR_UNSUPPORTED and "65535" in B.last_error()
 
 
 def test_workspace_size_is_counter_plus_scores():
