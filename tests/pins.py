@@ -309,3 +309,36 @@ def check_sparse_partition(rearrange, attend_problem, attend_full, merge):
         assert np.abs(a - a_ex).max() < 1e-12 and np.abs(l - l_ex).max() < 1e-12, "fresh partition is not exact"
     p2, kr, vr, ke, ve = rearrange(p, ko, vo, ki, vi, [[], []])
     assert np.array_equal(kr, ko) and np.array_equal(ve, vi) and np.array_equal(p2.cu_seqlens_kv_in, p.cu_seqlens_kv_in)
+
+
+# ---------------------------------------------------------------- branch hooks
+
+def check_branch_hooks(cache_copy_seq, cache_invalidate_seqs):
+    """BlockBatch, "Methodologie : BlockBatch", items 2 and 3.  Leader sync copies the
+    entries of the block positions both branches have, for every head, with the
+    leader's validity and count; a destination with more positions than the leader
+    stays empty; a refresh empties only the marked branches and restarts their
+    counts; nothing else changes."""
+    from cached_split_attention_b200.workloads import make_problem
+    from oracle import policy
+    p = make_problem([[0, 1, 2], [0, 1], [0, 1, 2, 3]], [5, 5, 5], [3, 2, 4], 2, 1, 4)
+    c = policy.OracleCache.empty(p)
+    rng = np.random.default_rng(0)
+    c.a_out[:] = rng.normal(size=c.a_out.shape)
+    c.l_out[:] = rng.normal(size=c.l_out.shape)
+    c.q_ref[:] = rng.normal(size=c.q_ref.shape)
+    c.valid[:] = [[True, False], [True, True], [False, True]]
+    c.m_acc[:] = [[1, 2], [3, 4], [5, 6]]
+    before = (c.a_out.copy(), c.l_out.copy(), c.q_ref.copy())
+    cache_copy_seq(c, p, 0, 1)          # B_src = 3 >= B_dst = 2
+    assert np.array_equal(c.a_out[3:5], before[0][0:2]) and np.array_equal(c.l_out[3:5], before[1][0:2])
+    assert np.array_equal(c.q_ref[3:5], before[2][0:2])
+    assert c.valid[1].tolist() == [True, False] and c.m_acc[1].tolist() == [1, 2]
+    assert np.array_equal(c.a_out[0:3], before[0][0:3]) and np.array_equal(c.a_out[5:], before[0][5:])
+    assert np.array_equal(c.l_out[0:3], before[1][0:3]) and np.array_equal(c.q_ref[0:3], before[2][0:3])
+    cache_copy_seq(c, p, 1, 2)          # B_src = 2 < B_dst = 4: dst cannot be filled
+    assert np.array_equal(c.a_out[5:7], before[0][0:2]) and np.array_equal(c.a_out[7:9], before[0][7:9])
+    assert not c.valid[2].any()
+    cache_invalidate_seqs(c, [True, False, False])
+    assert not c.valid[0].any() and c.m_acc[0].tolist() == [0, 0] and c.valid[1].tolist() == [True, False]
+    assert c.m_acc[1].tolist() == [1, 2]

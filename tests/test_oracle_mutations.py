@@ -145,6 +145,8 @@ def test_unmutated_oracle_passes_every_pin():
     pins.check_golden_gates(policy.decide)
     pins.check_cosine(policy.head_cosine)
     pins.check_problem_vs_brute(attention.attend_problem, attention.merge)
+    pins.check_cumulative_gate(policy.decide, policy.next_m_acc)
+    pins.check_branch_hooks(policy.cache_copy_seq, policy.cache_invalidate_seqs)
 
 
 SPARSE_MUTANTS = [
@@ -163,3 +165,31 @@ def test_sparse_mutants_caught(label, old, new):
     bad = mutate(sparse, "rearrange", old, new)
     assert caught(pins.check_sparse_partition, bad, attention.attend_problem, attention.attend_full,
                   attention.merge), label
+
+
+BRANCH_MUTANTS = [
+    ("copy: source and destination swapped", "cache.a_out[d0:d0 + n] = cache.a_out[s0:s0 + n]",
+     "cache.a_out[s0:s0 + n] = cache.a_out[d0:d0 + n]"),
+    ("copy: one position short", "n = min(s1 - s0, d1 - d0)", "n = min(s1 - s0, d1 - d0) - 1"),
+    ("copy: a longer destination marked valid", "cache.valid[dst] = cache.valid[src] & (d1 - d0 <= s1 - s0)",
+     "cache.valid[dst] = cache.valid[src]"),
+    ("copy: queries not copied", "cache.q_ref[d0:d0 + n] = cache.q_ref[s0:s0 + n]", "pass"),
+    ("copy: count not copied", "cache.m_acc[dst] = cache.m_acc[src]", "pass"),
+]
+
+REFRESH_MUTANTS = [
+    ("refresh: mask ignored", "cache.valid[m] = False", "cache.valid[:] = False"),
+    ("refresh: count kept", "cache.m_acc[m] = 0", "cache.m_acc[m] = cache.m_acc[m]"),
+]
+
+
+@pytest.mark.parametrize("label,old,new", BRANCH_MUTANTS, ids=[m[0] for m in BRANCH_MUTANTS])
+def test_branch_copy_mutants_caught(label, old, new):
+    bad = mutate(policy, "cache_copy_seq", old, new)
+    assert caught(pins.check_branch_hooks, bad, policy.cache_invalidate_seqs), label
+
+
+@pytest.mark.parametrize("label,old,new", REFRESH_MUTANTS, ids=[m[0] for m in REFRESH_MUTANTS])
+def test_refresh_mutants_caught(label, old, new):
+    bad = mutate(policy, "cache_invalidate_seqs", old, new)
+    assert caught(pins.check_branch_hooks, policy.cache_copy_seq, bad), label

@@ -96,23 +96,5 @@ def test_branch_hooks():
     """Leader sync copies a branch's entries (positions present on both sides, all
     heads) and its validity; a longer destination stays empty; a refresh empties
     only the marked branches; the other rows are untouched."""
-    from cached_split_attention_b200.workloads import make_problem
-    p = make_problem([[0, 1, 2], [0, 1], [0, 1, 2, 3]], [5, 5, 5], [3, 2, 4], 2, 1, 4)
-    c = policy.OracleCache.empty(p)
-    rng = np.random.default_rng(0)
-    c.a_out[:] = rng.normal(size=c.a_out.shape)
-    c.l_out[:] = rng.normal(size=c.l_out.shape)
-    c.q_ref[:] = rng.normal(size=c.q_ref.shape)
-    c.valid[:] = [[True, False], [True, True], [False, True]]
-    c.m_acc[:] = [[1, 2], [3, 4], [5, 6]]
-    before = (c.a_out.copy(), c.l_out.copy(), c.q_ref.copy())
-    policy.cache_copy_seq(c, p, 0, 1)          # B_src = 3 >= B_dst = 2
-    assert np.array_equal(c.a_out[3:5], before[0][0:2]) and np.array_equal(c.l_out[3:5], before[1][0:2])
-    assert np.array_equal(c.q_ref[3:5], before[2][0:2])
-    assert c.valid[1].tolist() == [True, False] and c.m_acc[1].tolist() == [1, 2]
-    assert np.array_equal(c.a_out[0:3], before[0][0:3]) and np.array_equal(c.a_out[5:], before[0][5:])
-    policy.cache_copy_seq(c, p, 1, 2)          # B_src = 2 < B_dst = 4: dst cannot be filled
-    assert np.array_equal(c.a_out[5:7], before[0][0:2]) and np.array_equal(c.a_out[7:9], before[0][7:9])
-    assert not c.valid[2].any()
-    policy.cache_invalidate_seqs(c, [True, False, False])
-    assert not c.valid[0].any() and c.m_acc[0].tolist() == [0, 0] and c.valid[1].tolist() == [True, False]
+    import pins
+    pins.check_branch_hooks(policy.cache_copy_seq, policy.cache_invalidate_seqs)
