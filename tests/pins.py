@@ -342,3 +342,93 @@ def check_branch_hooks(cache_copy_seq, cache_invalidate_seqs):
     cache_invalidate_seqs(c, [True, False, False])
     assert not c.valid[0].any() and c.m_acc[0].tolist() == [0, 0] and c.valid[1].tolist() == [True, False]
     assert c.m_acc[1].tolist() == [1, 2]
+
+
+# ---------------------------------------------------------------- the step policy
+
+def _replay_expected(w, flags):
+    """The FlashBlock policy restated without a cache: a head recomputes at the first
+    step and whenever its gate says so; the prefix partial it uses at step s is the
+    attention, over the prefix, of the queries it had at its last recompute (same
+    block positions); the output merges that with the attention of the current
+    queries over the current block (FlashBlock, "Mecanismo Central" and "Estrategias
+    de Reutilizacion Adaptativa")."""
+    from oracle import attention
+    from cached_split_attention_b200.workloads import GATE_HEAD, GATE_TAU, GATE_TAU_CUM
+    p0 = w.problem
+    S, H, Hk = p0.num_seqs, p0.num_heads_q, p0.num_heads_kv
+    g = H // Hk
+    last = np.full((S, H), -1)
+    count = np.zeros((S, H), dtype=np.int64)
+    qs, where = [], []   # per step: queries (fp64) and {(b, block position): packed row}
+    decisions, outs = [], []
+    for s, st in enumerate(w.steps):
+        p = st.problem
+        q = attention.bf16_to_f64(st.q)
+        qs.append(q)
+        where.append({(b, int(p.q_rows[r])): r for b in range(S)
+                      for r in range(int(p.cu_seqlens_q[b]), int(p.cu_seqlens_q[b + 1]))})
+        rec = np.zeros((S, H), dtype=bool)
+        for b in range(S):
+            r0, r1 = int(p.cu_seqlens_q[b]), int(p.cu_seqlens_q[b + 1])
+            n = int(st.n_updated[b])
+            for h in range(H):
+                if last[b, h] < 0:
+                    rec[b, h] = True
+                elif flags & GATE_TAU:
+                    rec[b, h] = n >= w.tau
+                elif flags & GATE_TAU_CUM:
+                    rec[b, h] = count[b, h] + n >= w.tau
+                elif flags & GATE_HEAD:
+                    then = [where[last[b, h]][(b, int(p.q_rows[r]))] for r in range(r0, r1)]
+                    x = q[r0:r1, h].ravel()
+                    y = qs[last[b, h]][then, h].ravel()
+                    den = math.sqrt(float(x @ x) * float(y @ y))
+                    cos = float(x @ y) / den if den > 0 else 0.0
+                    rec[b, h] = not (cos > w.gamma)
+            if flags & GATE_TAU_CUM:
+                count[b] = np.where(rec[b], 0, count[b] + n)
+        last[rec] = s
+        a_full = np.full((p.total_q, H, p.head_dim), np.nan)
+        l_full = np.full((p.total_q, H), np.nan)
+        for b in range(S):
+            r0, r1 = int(p.cu_seqlens_q[b]), int(p.cu_seqlens_q[b + 1])
+            if r1 == r0:
+                continue
+            o0, o1 = int(p.cu_seqlens_kv_out[b]), int(p.cu_seqlens_kv_out[b + 1])
+            i0, i1 = int(p.cu_seqlens_kv_in[b]), int(p.cu_seqlens_kv_in[b + 1])
+            for h in range(H):
+                then = [where[last[b, h]][(b, int(p.q_rows[r]))] for r in range(r0, r1)]
+                ko = attention.bf16_to_f64(w.k_out[o0:o1, h // g])
+                vo = attention.bf16_to_f64(w.v_out[o0:o1, h // g])
+                ki = attention.bf16_to_f64(st.k_in[i0:i1, h // g])
+                vi = attention.bf16_to_f64(st.v_in[i0:i1, h // g])
+                ao, lo = attention.attend(qs[last[b, h]][then, h], ko, vo, p.softmax_scale)
+                ai, li = attention.attend(q[r0:r1, h], ki, vi, p.softmax_scale)
+                a, l = attention.merge(ao, lo, ai, li)
+                a_full[r0:r1, h] = a
+                l_full[r0:r1, h] = l
+        decisions.append(rec)
+        outs.append((a_full, l_full))
+    return decisions, outs
+
+
+def check_policy_replay(run_policy):
+    """run_policy against the cache-free restatement above, on a cumulative-τ problem
+    with monotone locking (GQA), a τ-gated problem and a γ-gated problem: decisions
+    equal, outputs within 1e-12, and both reuse and recompute taken after step 0."""
+    from cached_split_attention_b200 import workloads as W
+    locking = W.locking_tiny()
+    locking.tau = 7       # 3 redraws per step: the count passes 7 at the third step
+    cases = [(locking, W.GATE_TAU_CUM),
+             (W.dllm_layer(steps=8, prefix=128), W.GATE_TAU),
+             (W.video(steps=4, block=48, prefix_blocks=2, heads=4, head_dim=64, sigma_lo=0.02, sigma_hi=0.6),
+              W.GATE_HEAD)]
+    for w, flags in cases:
+        got = run_policy(w, flags=flags)
+        dec, outs = _replay_expected(w, flags)
+        for s, (r, d, (a, l)) in enumerate(zip(got, dec, outs)):
+            assert np.array_equal(r.recompute, d), (w.name, s, "decisions")
+            _close(r.a_full, a, what=f"{w.name} step {s} A")
+            _close(r.l_full, l, what=f"{w.name} step {s} L")
+        assert any(d.any() for d in dec[1:]) and any((~d).any() for d in dec[1:]), (w.name, "both branches taken")

@@ -147,6 +147,7 @@ def test_unmutated_oracle_passes_every_pin():
     pins.check_problem_vs_brute(attention.attend_problem, attention.merge)
     pins.check_cumulative_gate(policy.decide, policy.next_m_acc)
     pins.check_branch_hooks(policy.cache_copy_seq, policy.cache_invalidate_seqs)
+    pins.check_policy_replay(policy.run_policy)
 
 
 SPARSE_MUTANTS = [
@@ -193,3 +194,19 @@ def test_branch_copy_mutants_caught(label, old, new):
 def test_refresh_mutants_caught(label, old, new):
     bad = mutate(policy, "cache_invalidate_seqs", old, new)
     assert caught(pins.check_branch_hooks, policy.cache_copy_seq, bad), label
+
+
+POLICY_MUTANTS = [
+    ("queries of a recompute not kept", "cache.q_ref[crow[rs_all], h] = q[rs_all, h]", "pass"),
+    ("cache written at the packed row", "cache.a_out[crow[rs], h] = a", "cache.a_out[rs, h] = a"),
+    ("a recompute never marks the entry valid", "cache.valid[b, h] = True", "pass"),
+    ("cumulative count not advanced", "cache.m_acc = next_m_acc(flags, cache.m_acc, st.n_updated, rec)", "pass"),
+    ("prefix of kv-head 0 for every head", "kk = bf16_to_f64(workload.k_out[o0:o1, hk])",
+     "kk = bf16_to_f64(workload.k_out[o0:o1, 0])"),
+]
+
+
+@pytest.mark.parametrize("label,old,new", POLICY_MUTANTS, ids=[m[0] for m in POLICY_MUTANTS])
+def test_policy_mutants_caught(label, old, new):
+    bad = mutate(policy, "run_policy", old, new)
+    assert caught(pins.check_policy_replay, bad), label

@@ -98,3 +98,11 @@ def test_branch_hooks():
     only the marked branches; the other rows are untouched."""
     import pins
     pins.check_branch_hooks(policy.cache_copy_seq, policy.cache_invalidate_seqs)
+
+
+def test_policy_equals_its_cache_free_restatement():
+    """run_policy equals the policy restated without a cache (each head's prefix
+    partial recomputed from the queries of its last recompute), under the
+    cumulative, per-step and similarity gates."""
+    import pins
+    pins.check_policy_replay(policy.run_policy)
