@@ -61,3 +61,12 @@ def test_varlen_offsets():
 def test_video_sigma_halves():
     w = W.video(steps=2, block=16, prefix_blocks=2, heads=8)
     assert (w.sigma < 0.1).sum() == 4 and w.flags == W.GATE_HEAD
+
+
+def test_dllm_default_recompute_steps():
+    """The 8B-dLLM layer as the bench runs it (seed 1001): with tau = 4 the steps
+    that recompute are 0, 2, 7, 12 and 25 (k = clamp(Poisson(2), 1, 4) reaches 4
+    at steps 2, 7, 12, 25)."""
+    w = W.dllm_layer()
+    ks = [int(s.n_updated[0]) for s in w.steps]
+    assert [0] + [s for s in range(1, 32) if ks[s] >= w.tau] == [0, 2, 7, 12, 25]
