@@ -347,11 +347,13 @@ def video(seed: int = 1004, steps: int = 10, block: int = 1560, prefix_blocks: i
 
 
 def locking_tiny(seed: int = 1010, steps: int = 5, block: int = 48, prefix: int = 96,
-                 heads_q: int = 4, heads_kv: int = 2, head_dim: int = 64) -> Workload:
+                 heads_q: int = 4, heads_kv: int = 2, head_dim: int = 64, redraws=(3, 3)) -> Workload:
     """SureLock-style monotone locking on a small GQA problem (two sequences).
 
     Every step locks a few more rows (the active set only shrinks), redraws the
-    Q/K/V of 3 still-active rows per sequence, and keeps tau gating on."""
+    Q/K/V of ``redraws[b]`` still-active rows of sequence b, and keeps tau gating
+    on (tau = 4: with the default 3 redraws both sequences reuse after step 0; with
+    (3, 5) the second sequence recomputes at every step and the first reuses)."""
     rng = np.random.default_rng(seed)
     active = [np.arange(block), np.arange(block - 8)]
     p0 = make_problem(active, [prefix, prefix + 37], [block, block - 8], heads_q, heads_kv, head_dim)
@@ -368,7 +370,7 @@ def locking_tiny(seed: int = 1010, steps: int = 5, block: int = 48, prefix: int 
         p = make_problem(active, [prefix, prefix + 37], [block, block - 8], heads_q, heads_kv, head_dim)
         toks = []
         for b, a in enumerate(active):
-            sel = rng.choice(a, size=min(3, len(a)), replace=False) + p.cu_seqlens_kv_in[b]
+            sel = rng.choice(a, size=min(int(redraws[b]), len(a)), replace=False) + p.cu_seqlens_kv_in[b]
             toks.append(np.sort(sel))
         st.redraw(np.concatenate(toks))
         out.append(st.step_input([len(t) for t in toks], p))

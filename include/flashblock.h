@@ -326,18 +326,22 @@ fb_status fb_device_status(int32_t* code, fb_stream_t stream);
  * holds the two-tile work order).  Larger problems return FB_ERR_UNSUPPORTED
  * (message in fb_noalloc_last_error()) -- use fb_step with a workspace for them.
  * No call allocates: the first call on a device resolves the scratch address
- * (cudaGetSymbolAddress), so make that first call before capturing a stream.
+ * (cudaGetSymbolAddress, with that device current), so make that first call before
+ * capturing a stream.  If the device's context is re-created (cudaDeviceReset), the
+ * next call resolves the address again, so that call too belongs before a capture.
  * Every call on a device shares the one array, which keeps the last call's
  * contents (the call clears the part that must start at zero): calls that could
  * overlap on the GPU race and must be ordered, e.g. issued on one stream.
- * Errors of argument checking are reported through fb_last_error().
+ * Every failure is described by fb_noalloc_last_error().
  */
 fb_status fb_step_noalloc(const fb_problem* problem, const fb_params* params, const fb_cache* cache,
                           const fb_bf16* q, const fb_bf16* k_in, const fb_bf16* v_in, const fb_bf16* k_out,
                           const fb_bf16* v_out, const int32_t* n_updated, const uint8_t* head_reuse_in,
                           fb_bf16* a_full, float* l_full, uint8_t* decision_out, fb_stream_t stream);
 
-/* Message of the last fb_step_noalloc failure that is not an argument error. */
+/* Message of the last fb_step_noalloc failure on this thread (every kind: argument
+ * errors, a problem above the scratch limit, CUDA errors); empty after a call that
+ * succeeded.  Argument errors are also reported through fb_last_error(). */
 const char* fb_noalloc_last_error(void);
 
 #ifdef __cplusplus

@@ -31,6 +31,24 @@ def _close(a, b, tol=TOL, what=""):
 
 # ---------------------------------------------------------------- definition
 
+def check_bf16_widening(bf16_to_f64):
+    """bf16 bit patterns widened to binary64 give the exact values the format
+    defines (tests/golden/bf16_bits.txt, derived by hand from the bit layout):
+    normals, the smallest subnormal, the largest finite value, signed zero, both
+    infinities and NaN; the shape of the input is kept."""
+    g = load("bf16_bits.txt")
+    bits = g["bits"].astype(np.uint16)
+    got = bf16_to_f64(bits)
+    assert got.dtype == np.float64, got.dtype
+    want = g["values"]
+    assert np.array_equal(got, want), (got, want)   # exact: widening must not round
+    two_d = bf16_to_f64(bits[:10].reshape(2, 5))
+    assert two_d.shape == (2, 5) and np.array_equal(two_d.reshape(-1), want[:10])
+    nz = bf16_to_f64(g["neg_zero_bits"].astype(np.uint16))
+    assert nz[0] == 0.0 and math.copysign(1.0, float(nz[0])) == -1.0, nz
+    assert np.isnan(bf16_to_f64(g["nan_bits"].astype(np.uint16))[0])
+
+
 def check_golden_attend(attend):
     for name in ("attend_two_keys.txt", "attend_three_keys_scaled.txt"):
         g = load(name)
@@ -309,6 +327,27 @@ def check_sparse_partition(rearrange, attend_problem, attend_full, merge):
         assert np.abs(a - a_ex).max() < 1e-12 and np.abs(l - l_ex).max() < 1e-12, "fresh partition is not exact"
     p2, kr, vr, ke, ve = rearrange(p, ko, vo, ki, vi, [[], []])
     assert np.array_equal(kr, ko) and np.array_equal(ve, vi) and np.array_equal(p2.cu_seqlens_kv_in, p.cu_seqlens_kv_in)
+
+
+def check_sparse_workload(sparse_workload, run_policy, attend_full):
+    """The sparse-residual workload, step by step: with FORCE_RECOMPUTE every step
+    merges a fresh residual partial (the prefix keys left out) with the partial over
+    the block and the selected keys, so at every step the result must be full
+    attention over prefix + block of that step's inputs (FlashBlock, "Estrategias de
+    Reutilizacion Adaptativa", third bullet, with "Mecanismo Central").  The block
+    K/V change at every step, so a rearrangement that kept an old block's keys
+    fails from step 1 on.  Run on the tiny workload (one sequence, sharp scores) and
+    on the locking workload (two sequences, GQA, shrinking active sets)."""
+    from cached_split_attention_b200 import workloads as W
+    cases = [(W.tiny(sharp=6.0, steps=4), [list(range(0, 16)) + [77, 130] + list(range(192, 256))]),
+             (W.locking_tiny(steps=3), [[0, 5, 6, 40, 95], list(range(20, 60))])]
+    for w, sel in cases:
+        assert any(not np.array_equal(st.k_in, w.steps[0].k_in) for st in w.steps[1:]), "block must change"
+        got = run_policy(sparse_workload(w, sel), flags=W.FORCE_RECOMPUTE)
+        for s, (r, st) in enumerate(zip(got, w.steps)):
+            a_ex, l_ex = attend_full(st.problem, st.q, w.k_out, w.v_out, st.k_in, st.v_in)
+            _close(r.a_full, a_ex, what=f"{w.name} sparse step {s} A")
+            _close(r.l_full, l_ex, what=f"{w.name} sparse step {s} L")
 
 
 # ---------------------------------------------------------------- branch hooks

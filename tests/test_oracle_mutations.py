@@ -148,6 +148,9 @@ def test_unmutated_oracle_passes_every_pin():
     pins.check_cumulative_gate(policy.decide, policy.next_m_acc)
     pins.check_branch_hooks(policy.cache_copy_seq, policy.cache_invalidate_seqs)
     pins.check_policy_replay(policy.run_policy)
+    pins.check_bf16_widening(attention.bf16_to_f64)
+    from oracle import sparse
+    pins.check_sparse_workload(sparse.sparse_workload, policy.run_policy, attention.attend_full)
 
 
 SPARSE_MUTANTS = [
@@ -210,3 +213,39 @@ POLICY_MUTANTS = [
 def test_policy_mutants_caught(label, old, new):
     bad = mutate(policy, "run_policy", old, new)
     assert caught(pins.check_policy_replay, bad), label
+
+
+WIDEN_MUTANTS = [
+    ("every value scaled by 1 + 2^-7", ".view(np.float32).astype(np.float64)",
+     ".view(np.float32).astype(np.float64) * (1 + 2.0 ** -7)"),
+    ("bits shifted by 15", "(b.astype(np.uint32) << 16)", "(b.astype(np.uint32) << 15)"),
+    ("widened through float16", "(b.astype(np.uint32) << 16).view(np.float32)",
+     "b.view(np.float16).astype(np.float32)"),
+    ("low fraction bit dropped", "b = np.ascontiguousarray(bits, dtype=np.uint16)",
+     "b = np.ascontiguousarray(bits, dtype=np.uint16) & np.uint16(0xFFFE)"),
+]
+
+
+@pytest.mark.parametrize("label,old,new", WIDEN_MUTANTS, ids=[m[0] for m in WIDEN_MUTANTS])
+def test_widen_mutants_caught(label, old, new):
+    bad = mutate(attention, "bf16_to_f64", old, new)
+    assert caught(pins.check_bf16_widening, bad), label
+
+
+SPARSE_WORKLOAD_MUTANTS = [
+    ("the first step's block on every step",
+     "rearrange(st.problem, workload.k_out, workload.v_out, st.k_in, st.v_in,",
+     "rearrange(st.problem, workload.k_out, workload.v_out, workload.steps[0].k_in, workload.steps[0].v_in,"),
+    ("the original prefix kept as the residual", "problem=p0, k_out=k_res, v_out=v_res,",
+     "problem=p0, k_out=workload.k_out, v_out=workload.v_out,"),
+    ("the step's queries replaced by step 0's", "steps.append(dataclasses.replace(st, k_in=k_ext, v_in=v_ext, problem=p2s))",
+     "steps.append(dataclasses.replace(st, q=workload.steps[0].q if workload.steps[0].q.shape == st.q.shape else st.q, "
+     "k_in=k_ext, v_in=v_ext, problem=p2s))"),
+]
+
+
+@pytest.mark.parametrize("label,old,new", SPARSE_WORKLOAD_MUTANTS, ids=[m[0] for m in SPARSE_WORKLOAD_MUTANTS])
+def test_sparse_workload_mutants_caught(label, old, new):
+    from oracle import sparse
+    bad = mutate(sparse, "sparse_workload", old, new)
+    assert caught(pins.check_sparse_workload, bad, policy.run_policy, attention.attend_full), label

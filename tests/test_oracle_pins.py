@@ -6,6 +6,10 @@ import pins
 from oracle import attention, policy
 
 
+def test_bf16_widening():
+    pins.check_bf16_widening(attention.bf16_to_f64)
+
+
 def test_golden_attend():
     pins.check_golden_attend(attention.attend)
 

@@ -3,11 +3,15 @@ import numpy as np
 
 import pins
 from cached_split_attention_b200 import workloads as W
-from oracle import attention, sparse
+from oracle import attention, policy, sparse
 
 
 def test_partition_pins():
     pins.check_sparse_partition(sparse.rearrange, attention.attend_problem, attention.attend_full, attention.merge)
+
+
+def test_sparse_workload_every_step_is_full_attention_when_recomputed():
+    pins.check_sparse_workload(sparse.sparse_workload, policy.run_policy, attention.attend_full)
 
 
 def test_sparse_policy_fresh_step_is_dense_and_reuse_is_closer():
