@@ -1,8 +1,13 @@
 """Benchmark of the FlashBlock denoise-step attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload dllm_layer|long_context_gqa|varlen_branches|video|tiny]
-                    [--layers L] [--rows]
+                    [--workload long_context_gqa|dllm_layer|varlen_branches|video|tiny]
+                    [--layers L] [--headline-only] [--rows]
+
+The headline workload (default: long-context GQA, the largest configuration:
+batch 8, prefix 32768, 1 GiB of prefix K/V per layer) gives the JSON line; on one
+GPU the other four configurations are then timed the same way and carried under
+"configs" of that line (--headline-only skips them).
 
 The workload is run the way a block-diffusion model runs it: every denoise step
 calls the attention of each of L layers (32 for the 8B dLLM), and every layer has
@@ -31,7 +36,8 @@ measured sustained bf16 tensor throughput; `roofline_all_launches` aggregates
 every launch.
 
 `--impl reference` times the fp64 oracle (the plain CPU statement of the method)
-on the host cores on one layer of the same workload, rank 0 only.
+on the host cores on one layer of the same workload, rank 0 only (for the
+long-context GQA batch: one of its 8 equal sequences, the time scaled by 8).
 
 `--rows` measures the extension rows instead (one JSON line, one GPU): the
 cumulative-M gate on the 8B-dLLM layer, the BlockBatch branch hooks on the
@@ -196,7 +202,7 @@ def make_workload(name: str, seed: int):
 
 # ---------------------------------------------------------------- native arm
 
-DEFAULT_LAYERS = {"dllm_layer": 32, "long_context_gqa": 2, "varlen_branches": 32, "video": 8, "tiny": 32}
+DEFAULT_LAYERS = {"dllm_layer": 32, "long_context_gqa": 32, "varlen_branches": 32, "video": 8, "tiny": 32}
 
 
 class Model:
@@ -382,18 +388,19 @@ def kernel_source_digest(kernel: str = "attn_kernel") -> str:
     return h.hexdigest()
 
 
-def native(args, world, rank, local):
+SEED_OF = {"tiny": 1000, "dllm_layer": 1001, "long_context_gqa": 1002, "varlen_branches": 1003, "video": 1004}
+# The configurations measured after the headline one in a default run (one GPU):
+# each gets its own line under "configs" of the same JSON object.
+EXTRA_ORDER = ("dllm_layer", "varlen_branches", "video", "tiny")
+
+
+def measure(name, args, world, rank, local, device):
+    """Time one workload as a model runs it (see the module docstring); returns the
+    JSON object of its line on rank 0 (None elsewhere)."""
     import torch
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    base = {"tiny": 1000, "dllm_layer": 1001, "long_context_gqa": 1002, "varlen_branches": 1003,
-            "video": 1004}[args.workload]
-    w = make_workload(args.workload, shard_seed(base, rank))
-    L = args.layers or DEFAULT_LAYERS[args.workload]
+    base = SEED_OF[name]
+    w = make_workload(name, shard_seed(base, rank))
+    L = (args.layers if name == args.workload else 0) or DEFAULT_LAYERS[name]
     model = Model(w, L, device)
     S = model.S
     p = w.problem
@@ -458,27 +465,23 @@ def native(args, world, rank, local):
     ach_rec = float(np.sum(bytes_rec) / np.sum(t_rec) / 1e9) if rec_steps else float("nan")
     bytes_all = sum(step_bytes(w.steps[s].problem, rec_frac[s])["total"] for s in range(S))
     ach_all = bytes_all / (episode_ms * 1e-3 / L) / 1e9
-    peaks = {}
-    try:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
-    except Exception:
-        pass
+    peaks = _peaks()
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
-    kernel = KERNEL_OF[args.workload]
+    kernel = KERNEL_OF[name]
     traffic = None
     try:
         prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
         for ent in prof.get("entries", []):
             # counters only count for the kernel source they were taken on
-            if (ent.get("workload") == args.workload and ent.get("kernel") == kernel
+            if (ent.get("workload") == name and ent.get("kernel") == kernel
                     and ent.get("kernel_source_sha256") == kernel_source_digest(kernel)):
                 traffic = ent.get("dram_bytes_per_recompute_launch")
     except Exception:
         pass
     # the video block is a dense contraction (about 1500 flop per byte): its bound
     # is the tensor cores, timed inside a long step (the sustained bf16 figure)
-    tensor_bound = args.workload == "video"
+    tensor_bound = name == "video"
     flops_rec = [step_flops(w.steps[s].problem, rec_frac[s]) for s in rec_steps]
     ach_tf = float(np.sum(flops_rec) / np.sum(t_rec) / 1e12) if rec_steps else float("nan")
     tf_peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
@@ -488,21 +491,17 @@ def native(args, world, rank, local):
     e2e_v = max_over_ranks(e2e_call_us, world, device)
     ms_step = max_over_ranks(episode_ms, world, device)
     clocks = sampler.summary()
+    del model
+    torch.cuda.empty_cache()
     if rank != 0:
-        _teardown(world)
-        return
+        return None
 
     dense_b = step_bytes(p, 1.0)["total"]
     reuse_b = step_bytes(p, 0.0)["total"]
     dense_med = float(np.median(dense_us))
     reuse_med = float(np.median(reuse_us))
-    # kernels per call: the attention kernel; the similarity kernel under the gamma
-    # gate; the work-order pass when the two-tile kernel runs with the gates on
-    gated = not (w.flags & (W.FORCE_RECOMPUTE | W.FORCE_REUSE))
-    two_tile = p.head_dim == 128 and p.num_heads_q == p.num_heads_kv and p.max_q >= 256
-    per_call = 1 + (1 if gated and w.flags & W.GATE_HEAD else 0) + (1 if gated and two_tile else 0)
-    n_launch = args.steps * S * L * per_call
-    out = {
+    n_launch = args.steps * L * sum(launches_per_call(w, s) for s in range(S))
+    return {
         "metric": METRIC,
         "value": round(value, 3),
         "unit": "us/attention-call (one layer, one denoise step)",
@@ -516,7 +515,7 @@ def native(args, world, rank, local):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {
-            "workload": WORKLOAD_DESC[args.workload],
+            "workload": WORKLOAD_DESC[name],
             "layers": L,
             "bench_step": f"one denoise episode: {S} denoise steps x {L} layers = {S * L} fb_step calls",
             "recompute_steps_per_episode": len(rec_steps),
@@ -533,7 +532,8 @@ def native(args, world, rank, local):
                           "tflops": round(step_flops(p, 1.0) / dense_med / 1e6, 1)},
         "reuse_call_us": {"median": round(reuse_med, 3), "p10": round(float(np.percentile(reuse_us, 10)), 3),
                           "p90": round(float(np.percentile(reuse_us, 90)), 3),
-                          "effective_tbps": round(reuse_b / reuse_med / 1e6, 3)},
+                          "effective_tbps": round(reuse_b / reuse_med / 1e6, 3),
+                          "frac_of_hbm": round(reuse_b / reuse_med / 1e3 / hbm_peak, 4)},
         "reuse_gain": {"predicted_bytes_ratio": round(dense_b / reuse_b, 2),
                        "achieved_time_ratio": round(dense_med / reuse_med, 2)},
         "roofline": dict(
@@ -555,8 +555,49 @@ def native(args, world, rank, local):
         "gpu_launches": int(n_launch),
         "clocks": clocks,
     }
+
+
+def launches_per_call(w, s: int) -> int:
+    """Kernels one fb_step call of step s launches: the attention kernel; the
+    similarity kernel under the gamma gate; the work-order pass when the two-tile
+    kernel runs with the gates on."""
+    p = w.steps[s].problem
+    gated = not (w.flags & (W.FORCE_RECOMPUTE | W.FORCE_REUSE))
+    two_tile = p.head_dim == 128 and p.num_heads_q == p.num_heads_kv and p.max_q >= 256
+    return 1 + (1 if gated and w.flags & W.GATE_HEAD else 0) + (1 if gated and two_tile else 0)
+
+
+def config_summary(line: dict) -> dict:
+    """The keys of a configuration's line carried under "configs" of the headline."""
+    keys = ("value", "unit", "ms_per_step", "dense_call_us", "reuse_call_us", "reuse_gain", "roofline", "e2e",
+            "gpu_launches", "clocks")
+    out = {k: line[k] for k in keys}
+    out["config"] = {k: line["config"][k] for k in ("workload", "layers", "bench_step", "recompute_steps_per_episode",
+                                                    "seed")}
+    return out
+
+
+def native(args, world, rank, local):
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    out = measure(args.workload, args, world, rank, local, device)
+    # the other configurations, one GPU only (their lines ride along under "configs")
+    extra = [n for n in EXTRA_ORDER if n != args.workload] if (world == 1 and not args.headline_only) else []
+    if extra and rank == 0:
+        out["configs"] = {}
+        for name in extra:
+            out["configs"][name] = config_summary(measure(name, args, world, rank, local, device))
+    if rank != 0:
+        _teardown(world)
+        return
     if world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.workload, shard_seed(base, rank), budget_s=args.cpu_budget)
+        out["cpu_baseline"] = cpu_baseline(args.workload, shard_seed(SEED_OF[args.workload], rank),
+                                           budget_s=args.cpu_budget)
     print(json.dumps(out), flush=True)
     _teardown(world)
 
@@ -883,11 +924,24 @@ def host_cpu() -> dict:
     return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
+def oracle_sample(name: str, seed: int):
+    """The workload the CPU oracle times and the factor that scales its time to one
+    full attention call: the long-context GQA batch is 8 sequences of the same
+    shape, so one of them is timed and the time multiplied by 8; the other
+    workloads are timed whole."""
+    w = make_workload(name, seed)
+    if name == "long_context_gqa":
+        n = w.problem.num_seqs
+        return W.first_sequences(w, 1), float(n), f"1 of the {n} sequences (same shape), time x {n}"
+    return w, 1.0, "every sequence"
+
+
 def cpu_baseline(workload: str, seed: int, budget_s: float = 12.0) -> dict:
     """The fp64 oracle (as it stands) on a bounded sample: whole episodes of the
-    same workload until about budget_s seconds have passed."""
+    same workload (one sequence of a batch of equal sequences, scaled) until about
+    budget_s seconds have passed."""
     from oracle import policy
-    w = make_workload(workload, seed)
+    w, scale, what = oracle_sample(workload, seed)
     S = len(w.steps)
     t0 = time.perf_counter()
     n = 0
@@ -897,18 +951,17 @@ def cpu_baseline(workload: str, seed: int, budget_s: float = 12.0) -> dict:
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": round(dt / (n * S) * 1e6, 1), "unit": "us/attention-call (one layer, one denoise step)",
+    return {"value": round(dt / (n * S) * scale * 1e6, 1), "unit": "us/attention-call (one layer, one denoise step)",
             "cores": _oracle_threads(), "host": host_cpu(), "kind": "oracle",
-            "sample": f"{n} full episode(s) of {S} denoise steps of one layer, every row and head, fp64 numpy"}
+            "sample": f"{n} full episode(s) of {S} denoise steps of one layer, {what}, every row and head, "
+                      f"fp64 numpy"}
 
 
 def reference(args, world, rank):
     if rank != 0:
         return
     from oracle import policy
-    base = {"tiny": 1000, "dllm_layer": 1001, "long_context_gqa": 1002, "varlen_branches": 1003,
-            "video": 1004}[args.workload]
-    w = make_workload(args.workload, shard_seed(base, 0))
+    w, scale, what = oracle_sample(args.workload, shard_seed(SEED_OF[args.workload], 0))
     S = len(w.steps)
     for _ in range(args.warmup):
         policy.run_policy(w)
@@ -916,7 +969,7 @@ def reference(args, world, rank):
     for _ in range(args.steps):
         policy.run_policy(w)
     dt = time.perf_counter() - t0
-    us = dt / (args.steps * S) * 1e6
+    us = dt / (args.steps * S) * scale * 1e6
     cores = _oracle_threads()
     out = {
         "impl": "reference",
@@ -926,7 +979,7 @@ def reference(args, world, rank):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "ms_per_step": round(dt / args.steps * scale * 1e3, 3),
         "higher_is_better": False,
         "scaling": "weak",
         "vs_baseline": None,
@@ -936,7 +989,8 @@ def reference(args, world, rank):
                    "bench_step": f"one denoise episode ({S} steps) of one layer, fp64 oracle on host cores"},
         "cpu_baseline": {"value": round(us, 1), "unit": "us/attention-call (one layer, one denoise step)",
                          "cores": cores, "host": host_cpu(), "kind": "oracle",
-                         "sample": f"{args.steps} full episode(s) of {S} denoise steps of one layer, every row and head"},
+                         "sample": f"{args.steps} full episode(s) of {S} denoise steps of one layer, {what}, "
+                                   f"every row and head"},
         "e2e": {"value": round(us, 1), "unit": "us/attention-call (one layer, one denoise step)",
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -949,7 +1003,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=sorted(WORKLOAD_DESC), default="dllm_layer")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_DESC), default="long_context_gqa")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only --workload (by default one GPU also times the other four configurations)")
     ap.add_argument("--layers", type=int, default=0, help="attention layers per denoise step (0: workload default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

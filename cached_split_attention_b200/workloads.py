@@ -378,6 +378,27 @@ def locking_tiny(seed: int = 1010, steps: int = 5, block: int = 48, prefix: int 
                     notes="2 seqs, GQA 4/2, d64, monotone locking, 3 redraws/step")
 
 
+def first_sequences(w: Workload, n: int) -> Workload:
+    """The same workload restricted to its first ``n`` sequences (input slicing only:
+    the index arrays, Q rows, block and prefix K/V and update counts of those
+    sequences).  Used to time the CPU oracle on a bounded sample of a batch whose
+    sequences all have the same shape."""
+    def cut(p: Problem) -> Problem:
+        return Problem(num_seqs=n, num_heads_q=p.num_heads_q, num_heads_kv=p.num_heads_kv, head_dim=p.head_dim,
+                       softmax_scale=p.softmax_scale, cu_seqlens_q=p.cu_seqlens_q[:n + 1].copy(),
+                       q_rows=p.q_rows[:int(p.cu_seqlens_q[n])].copy(),
+                       cu_seqlens_kv_out=p.cu_seqlens_kv_out[:n + 1].copy(),
+                       cu_seqlens_kv_in=p.cu_seqlens_kv_in[:n + 1].copy())
+    p0 = cut(w.problem)
+    steps = []
+    for st in w.steps:
+        p = cut(st.problem)
+        steps.append(StepInput(q=st.q[:p.total_q], k_in=st.k_in[:p.total_kv_in], v_in=st.v_in[:p.total_kv_in],
+                               n_updated=st.n_updated[:n].copy(), problem=p))
+    return dataclasses.replace(w, problem=p0, k_out=w.k_out[:p0.total_kv_out], v_out=w.v_out[:p0.total_kv_out],
+                               steps=steps)
+
+
 NAMED = {
     "tiny": tiny,
     "dllm_layer": dllm_layer,

@@ -87,3 +87,20 @@ def test_cpu_baseline_reports_its_host():
     assert out["kind"] == "oracle" and out["value"] > 0 and out["cores"] >= 1
     assert out["host"]["nproc"] == os.cpu_count()
     assert out["host"]["cpu_model"] is None or isinstance(out["host"]["cpu_model"], str)
+
+
+def test_oracle_sample_of_the_gqa_batch_is_its_first_sequence():
+    """The CPU legs time one of the long-context batch's equal sequences and scale by
+    the batch size: the sample must be exactly sequence 0 of the batch (same rows,
+    keys and decisions as in the whole batch)."""
+    from cached_split_attention_b200 import workloads as W
+    from oracle import policy
+    w = W.long_context_gqa(steps=3, prefix=96, batch=3)
+    one = W.first_sequences(w, 1)
+    assert one.problem.num_seqs == 1 and one.problem.total_kv_out == 96
+    full = policy.run_policy(w)
+    part = policy.run_policy(one)
+    for f, p in zip(full, part):
+        n = p.problem.total_q
+        assert np.array_equal(f.recompute[:1], p.recompute)
+        assert np.array_equal(f.a_full[:n], p.a_full) and np.array_equal(f.l_full[:n], p.l_full)
