@@ -560,10 +560,12 @@ def measure(name, args, world, rank, local, device):
 def launches_per_call(w, s: int) -> int:
     """Kernels one fb_step call of step s launches: the attention kernel; the
     similarity kernel under the gamma gate; the work-order pass when the two-tile
-    kernel runs with the gates on."""
+    kernel runs with the gates on (from the library's own plan)."""
+    from cached_split_attention_b200 import binding as B
     p = w.steps[s].problem
     gated = not (w.flags & (W.FORCE_RECOMPUTE | W.FORCE_REUSE))
-    two_tile = p.head_dim == 128 and p.num_heads_q == p.num_heads_kv and p.max_q >= 256
+    plan = B.plan_query(B.DeviceProblem(p, "cpu"), B.CALL_STEP)
+    two_tile = plan["kernel_name"] == "tc2_attn_kernel"
     return 1 + (1 if gated and w.flags & W.GATE_HEAD else 0) + (1 if gated and two_tile else 0)
 
 

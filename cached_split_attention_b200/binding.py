@@ -55,7 +55,8 @@ class FbParams(ctypes.Structure):
 
 class FbPlanInfo(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("kernel", "rows_per_tile", "tiles", "work_items", "splits", "ctas",
-                                              "threads", "smem_bytes", "keys_per_chunk", "num_sms")]
+                                              "threads", "smem_bytes", "keys_per_chunk", "num_sms",
+                                              "lean_reuse", "lean_smem_bytes")]
 
 
 def _load():
@@ -80,6 +81,7 @@ def _load():
         "fb_cache_copy_seq": (st, [P, ctypes.POINTER(FbCache), ctypes.c_int32, ctypes.c_int32, vp]),
         "fb_cache_invalidate_seqs": (st, [P, ctypes.POINTER(FbCache), vp, vp]),
         "fb_sparse_layout": (st, [P, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "fb_prefix_append": (st, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "fb_selftest_wait_timeout": (st, [vp]),
         "fb_release_cache": (st, []),
         "fb_device_status": (st, [ctypes.POINTER(ctypes.c_int32), vp]),
@@ -260,6 +262,13 @@ def sparse_layout(problem: DeviceProblem, cu_sel, sel_idx, total_sel: int, k_out
     _check(_lib.fb_sparse_layout(problem.ref, _ptr(cu_sel), _ptr(sel_idx), int(total_sel), _ptr(k_out), _ptr(v_out),
                                  _ptr(k_in), _ptr(v_in), _ptr(k_res), _ptr(v_res), _ptr(k_ext), _ptr(v_ext),
                                  _ptr(cu_out_res), _ptr(cu_in_ext), _stream(stream)))
+
+
+def prefix_append(problem: DeviceProblem, k_out, v_out, k_in, v_in, k_dst, v_dst, cu_out_dst=None, stream=None):
+    """fb_prefix_append: block transition -- each sequence's finished block K/V follow
+    its prefix in (k_dst, v_dst) (see flashblock.h)."""
+    _check(_lib.fb_prefix_append(problem.ref, _ptr(k_out), _ptr(v_out), _ptr(k_in), _ptr(v_in), _ptr(k_dst),
+                                 _ptr(v_dst), _ptr(cu_out_dst), _stream(stream)))
 
 
 def selftest_wait_timeout(stream=None):

@@ -17,6 +17,7 @@
 #include "fb_selftest.cuh"
 #include "fb_sparse.cuh"
 #include "fb_tc2_kernel.cuh"
+#include "fb_transition.cuh"
 #include "flashblock.h"
 
 namespace {
@@ -96,6 +97,9 @@ struct Plan {
   int bn = fb::kBN;  // keys per pipeline chunk (TMA box rows)
   size_t off_grid_ctr = 0, off_cos = 0, off_order = 0, bytes = 0;
   int order_items = 0;  // work items of the two-tile kernel (0: the problem never takes it)
+  // lean reuse path (fused step, blocks of at most reuse::kMaxKeys keys)
+  bool reuse = false;
+  int reuse_chunks = 0, reuse_smem = 0;
 };
 
 int device_sms() {
@@ -191,6 +195,17 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = fals
     splits = std::max(1, std::min({splits, fb::kMaxSplits, chunks}));
   }
   pl.splits = splits;
+  // Lean reuse path: blocks of up to 128 keys, when the kernel's shared memory
+  // holds the block K/V and a tile of rows with their cache entries.
+  if (fused && !pl.tc2 && p->max_kv_in > 0 && p->max_kv_in <= fb::reuse::kMaxKeys) {
+    const int chunks = (p->max_kv_in + fb::kBN - 1) / fb::kBN;
+    const int need = fb::reuse::smem_bytes(pl.d, chunks, (pl.tr + 15) / 16 * 16) + 1024;
+    if (need <= pl.smem) {
+      pl.reuse = true;
+      pl.reuse_chunks = chunks;
+      pl.reuse_smem = need;
+    }
+  }
   // workspace layout
   size_t off = 0;
   pl.off_grid_ctr = off;
@@ -375,6 +390,8 @@ fb_status fb_plan_query(const fb_problem* problem, int32_t call, fb_plan_info* o
   out->smem_bytes = pl.smem;
   out->keys_per_chunk = pl.bn;
   out->num_sms = sms;
+  out->lean_reuse = pl.reuse ? 1 : 0;
+  out->lean_smem_bytes = pl.reuse ? pl.reuse_smem : 0;
   return FB_OK;
 }
 
@@ -547,6 +564,12 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   prm.a_full = reinterpret_cast<__nv_bfloat16*>(a_full);
   prm.l_full = l_full;
   prm.decision_out = decision_out;
+  if (pl.reuse) {
+    prm.k_in = reinterpret_cast<const __nv_bfloat16*>(k_in);
+    prm.v_in = reinterpret_cast<const __nv_bfloat16*>(v_in);
+    prm.reuse_chunks = pl.reuse_chunks;
+    prm.lean = 1;
+  }
   if (order_work) {
     int* order = reinterpret_cast<int*>(static_cast<char*>(workspace) + pl.off_order);
     if (pl.n_groups != pl.order_items)
@@ -648,6 +671,50 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
   void* args[] = {&sp};
   cudaError_t e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&fb::sparse_layout_kernel), args);
   if (e != cudaSuccess) return cuda_fail(e, "sparse layout kernel launch");
+  return FB_OK;
+}
+
+fb_status fb_prefix_append(const fb_problem* problem, const fb_bf16* k_out, const fb_bf16* v_out,
+                           const fb_bf16* k_in, const fb_bf16* v_in, fb_bf16* k_dst, fb_bf16* v_dst,
+                           int32_t* cu_seqlens_kv_out_dst, fb_stream_t stream) {
+  FB_TRY(check_problem(problem));
+  if (problem->num_seqs == 0) return FB_OK;
+  if (problem->num_seqs > 65535)  // one grid row per sequence
+    return fail(FB_ERR_UNSUPPORTED, "fb_prefix_append takes at most 65535 sequences per call");
+  const bool in_place = k_dst == k_out && problem->total_kv_out > 0;
+  if (in_place != (v_dst == v_out && problem->total_kv_out > 0))
+    return fail(FB_ERR_INVALID_ARG, "K and V must both be appended in place or both into new buffers");
+  if (in_place && problem->num_seqs != 1)
+    return fail(FB_ERR_UNSUPPORTED, "in-place append takes one sequence (later sequences would have to move)");
+  const long grown = static_cast<long>(problem->total_kv_out) + problem->total_kv_in;
+  if (grown >= (1L << 31)) return fail(FB_ERR_UNSUPPORTED, "grown prefix of %ld tokens", grown);
+  FB_TRY(check_ptr(k_out, "k_out", problem->total_kv_out > 0));
+  FB_TRY(check_ptr(v_out, "v_out", problem->total_kv_out > 0));
+  FB_TRY(check_ptr(k_in, "k_in", problem->total_kv_in > 0));
+  FB_TRY(check_ptr(v_in, "v_in", problem->total_kv_in > 0));
+  FB_TRY(check_ptr(k_dst, "k_dst", grown > 0));
+  FB_TRY(check_ptr(v_dst, "v_dst", grown > 0));
+  fb::AppendParams ap{problem->num_seqs, problem->num_heads_kv, problem->head_dim, problem->total_kv_out,
+                      problem->total_kv_in, in_place ? 0 : 1, problem->cu_seqlens_kv_out, problem->cu_seqlens_kv_in,
+                      reinterpret_cast<const __nv_bfloat16*>(k_out), reinterpret_cast<const __nv_bfloat16*>(v_out),
+                      reinterpret_cast<const __nv_bfloat16*>(k_in), reinterpret_cast<const __nv_bfloat16*>(v_in),
+                      reinterpret_cast<__nv_bfloat16*>(k_dst), reinterpret_cast<__nv_bfloat16*>(v_dst),
+                      cu_seqlens_kv_out_dst};
+  const long per_seq = static_cast<long>((in_place ? 0 : problem->max_kv_out) + problem->max_kv_in) *
+                       problem->num_heads_kv * problem->head_dim / 8;
+  const int bx = static_cast<int>(std::max<long>(1, std::min<long>((per_seq + 255) / 256, 1184)));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(bx, problem->num_seqs);
+  cfg.blockDim = dim3(256);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* args[] = {&ap};
+  cudaError_t e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&fb::prefix_append_kernel), args);
+  if (e != cudaSuccess) return cuda_fail(e, "prefix append kernel launch");
   return FB_OK;
 }
 

@@ -87,6 +87,11 @@ struct alignas(64) Params {
   // workspace
   int* grid_ctr;     // completion counter of the cache-state epilogue (zero between calls)
   const int* order;  // work order of the two-tile kernel (NULL: CTA i takes item i)
+  // lean reuse path (fb_reuse.cuh)
+  const __nv_bfloat16* k_in;  // block K/V, plain pointers
+  const __nv_bfloat16* v_in;
+  int reuse_chunks;  // 64-key chunks of the longest block
+  int lean;          // 1: groups whose heads all reuse take the lean path
 };
 
 // Reuse decision of (b, h); see fb_step in flashblock.h.
@@ -379,6 +384,12 @@ __device__ __forceinline__ void consume_keys(Acc<D>& acc, const uint32_t (&qf)[D
   }
 }
 
+}  // namespace fb
+
+#include "fb_reuse.cuh"  // the lean reuse path (uses the helpers above)
+
+namespace fb {
+
 template <int D, int WM, int WN, int STAGES>
 __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kernel(const __grid_constant__ Params p) {
   pdl_wait();
@@ -453,8 +464,17 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
 
   // decisions of this group's heads (written once per (b, kv-head))
   if (p.decision_out && t == 0 && split == S - 1 && tid < g) p.decision_out[b * p.hq + hk * g + tid] = s_rec[tid];
-
-  if (active && (has_in || has_out || cluster_mode)) {
+  // A group whose heads all reuse takes the lean reuse path (its CTAs share the rows).
+  const bool lean = p.lean && !any_rec && active;
+  if (lean) {
+    int r0, nr;
+    lean_rows(nrows, split, S, r0, nr);
+    if (n_in > p.reuse_chunks * kBN) {
+      if (tid == 0) record_status(kDevBadIndex);
+    } else if (nr > 0) {
+      lean_reuse<D>(p, smem, b, hk, q0, in0, n_in, row0 + r0, nr, tid, C::kThreads);
+    }
+  } else if (active && (has_in || has_out || cluster_mode)) {
     // -------------------------------------------------------- Q rows first
     // (before the K/V flood, so their loads are not queued behind it)
     constexpr int kQVec = TR * (D / 8);

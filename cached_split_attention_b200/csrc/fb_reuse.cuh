@@ -1,0 +1,185 @@
+// Lean reuse path of the fused FlashBlock step (sm_100a).
+//
+// On a reuse step the out-of-block partial (A_out, L_out) comes from the cache, so
+// the only attention left is the block's own: every active query row against the
+// block's B keys (bidirectional), followed by the log-space merge with the cached
+// row (FlashBlock, "Mecanismo Central": the stored values are reused instead of
+// reading the prefix K/V again).  That is a few MB per call and a short chain of
+// dependent loads, so when no head of a group (sequence, kv-head, row tile)
+// recomputes, the streaming kernels hand the group to this path instead of their
+// TMA pipeline, cluster and merge phases.  The group's CTAs share its rows (16 per
+// warp) and each runs:
+//
+//   loads      Q rows, the block K/V of the kv-head and q_rows, all issued together
+//              as 16-byte cp.async into shared memory; then the cached A_out /
+//              L_out rows at the rows' block positions;
+//   attention  S = Q K^T and O = P V with mma.sync (bf16 in, fp32 accumulate),
+//              online softmax in base 2 (the streaming kernel's inner loop);
+//   merge      in registers: A_full = w_out A_out + w_in A_in, L_full =
+//              logaddexp(L_out, L_in), written as bf16 / fp32.
+//
+// K and V sit in shared memory in the 128-byte swizzled layout of the warp-MMA
+// kernel's stages (64-key chunks), so the same inner loop serves both.  Keys past
+// the block's end are zero-filled and masked.  Blocks of up to kMaxKeys keys take
+// this path (the host plan checks max_kv_in and the shared memory it needs);
+// longer blocks are real contractions and stay on the streaming pipelines.
+//
+// Included by fb_kernels.cuh after the helpers it shares with the warp-MMA kernel
+// (Params, swz, Acc, consume_keys) and before the kernels that call it.
+#pragma once
+
+namespace fb {
+namespace reuse {
+
+constexpr int kMaxKeys = 128;  // block keys a CTA holds: two 64-key chunks
+
+// Shared memory of the lean path for `chunks` 64-key chunks and `rows` rows (a
+// multiple of 16), after the 1024-byte alignment of the kernel's base.
+__host__ __device__ constexpr int tile_bytes(int d) { return kBN * d * 2; }
+__host__ __device__ constexpr int q_stride(int d) { return d + 8; }  // padded bf16 Q row
+__host__ __device__ constexpr int c_stride(int d) { return d + 4; }  // padded fp32 cache row
+__host__ __device__ constexpr int smem_bytes(int d, int chunks, int rows) {
+  return 2 * chunks * tile_bytes(d) + rows * q_stride(d) * 2 + rows * c_stride(d) * 4 + rows * 4 + rows * 4;
+}
+
+}  // namespace reuse
+
+// Rows [r0, r0 + nr) of group (b, hk) -- row rho = (token rho / g, q-head hk*g +
+// rho % g) of the sequence's packed active tokens -- with the block keys of b.
+// Every thread of the CTA calls it (it has CTA barriers); `smem` is the kernel's
+// 1024-byte aligned dynamic shared memory.
+template <int D>
+__device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b, int hk, int q0, int in0, int n_in,
+                                           int r0, int nr, int tid, int nthreads) {
+  constexpr int kVec = D / 8;   // 16-byte vectors of a bf16 row
+  constexpr int kCVec = D / 4;  // 16-byte vectors of an fp32 row
+  constexpr int kT = reuse::tile_bytes(D);
+  constexpr int kQS = reuse::q_stride(D);
+  constexpr int kCS = reuse::c_stride(D);
+  const int g = p.g;
+  const int nch = p.reuse_chunks;
+  const int nr16 = (nr + 15) & ~15;
+  uint8_t* ks = smem;
+  uint8_t* vs = smem + nch * kT;
+  __nv_bfloat16* q_s = reinterpret_cast<__nv_bfloat16*>(smem + 2 * nch * kT);
+  float* ca_s = reinterpret_cast<float*>(smem + 2 * nch * kT + nr16 * kQS * 2);
+  float* cl_s = ca_s + nr16 * kCS;
+  int* pos_s = reinterpret_cast<int*>(cl_s + nr16);
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // Block K/V of kv-head hk: key rows up to the next multiple of 32 (the MMA's key
+  // slice); rows past the block's end are zero (masked scores, zero values).
+  const int n_keys = (n_in + 31) & ~31;
+  for (int it = tid; it < 2 * n_keys * kVec; it += nthreads) {
+    const int is_v = it >= n_keys * kVec;
+    const int v = is_v ? it - n_keys * kVec : it;
+    const int kr = v / kVec;
+    const int c = v % kVec;
+    uint8_t* dst = (is_v ? vs : ks) + (kr / kBN) * kT + swz(kr % kBN, c * 8);
+    if (kr < n_in) {
+      const __nv_bfloat16* src = (is_v ? p.v_in : p.k_in) + (static_cast<size_t>(in0 + kr) * p.hkv + hk) * D + c * 8;
+      cp_async_16(dst, src);
+    } else {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  for (int it = tid; it < nr16 * kVec; it += nthreads) {
+    const int r = it / kVec;
+    const int c = it % kVec;
+    __nv_bfloat16* dst = q_s + r * kQS + c * 8;
+    if (r < nr) {
+      const int rho = r0 + r;
+      cp_async_16(dst, p.q + (static_cast<size_t>(q0 + rho / g) * p.hq + hk * g + rho % g) * D + c * 8);
+    } else {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  cp_async_commit();
+  for (int r = tid; r < nr16; r += nthreads) {
+    int pos = -1;
+    if (r < nr) {
+      const int rho = r0 + r;
+      pos = p.q_rows ? p.q_rows[q0 + rho / g] : rho / g;
+      if (pos < 0 || pos >= n_in) {
+        record_status(kDevBadIndex);
+        pos = -1;
+      }
+    }
+    pos_s[r] = pos;
+  }
+  __syncthreads();
+  // cached rows at the block positions
+  for (int it = tid; it < nr * (kCVec + 1); it += nthreads) {
+    const int r = it / (kCVec + 1);
+    const int c = it % (kCVec + 1);
+    const int pos = pos_s[r];
+    if (pos < 0) continue;
+    const size_t ce = static_cast<size_t>(in0 + pos) * p.hq + hk * g + (r0 + r) % g;
+    if (c < kCVec) {
+      cp_async_16(ca_s + r * kCS + c * 4, p.cache_a + ce * D + c * 4);
+    } else {
+      cp_async_4(cl_s + r, p.cache_l + ce);
+    }
+  }
+  cp_async_commit();
+  cp_async_wait_all();
+  __syncthreads();
+
+  for (int slab = warp; slab * 16 < nr; slab += nthreads / 32) {
+    uint32_t qf[D / 16][4];
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      ldsm_x4(qf[kk], smem_u32(q_s + (16 * slab + (lane & 15)) * kQS + kk * 16 + (lane >> 4) * 8));
+    Acc<D> acc;
+    acc.reset();
+    for (int k0 = 0; k0 < n_keys; k0 += 32) {
+      const uint32_t kb = smem_u32(ks + (k0 / kBN) * kT);
+      const uint32_t vb = smem_u32(vs + (k0 / kBN) * kT);
+      consume_keys<D, 32>(acc, qf, kb, vb, k0 % kBN, k0, n_in, p.scale_log2, lane);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float z = quad_sum(acc.l[i]);
+      const int r = 16 * slab + (lane >> 2) + 8 * i;
+      if (r >= nr || pos_s[r] < 0) continue;
+      const int rho = r0 + r;
+      const size_t fe = static_cast<size_t>(q0 + rho / g) * p.hq + hk * g + rho % g;
+      const float li2 = z > 0.f ? acc.m[i] + lg2_approx(z) : kNegInf;
+      const float lo_nat = cl_s[r];
+      const float lo2 = lo_nat == kNegInf ? kNegInf : lo_nat * kLog2e;
+      const float m2 = fmaxf(lo2, li2);
+      float wo = 0.f, wi = 0.f, lf2 = kNegInf;
+      if (m2 != kNegInf) {
+        wo = lo2 == kNegInf ? 0.f : ex2(lo2 - m2);
+        wi = li2 == kNegInf ? 0.f : ex2(li2 - m2);
+        const float inv = rcp_approx(wo + wi);
+        lf2 = m2 + lg2_approx(wo + wi);
+        wo *= inv;
+        wi *= inv;
+      }
+      const float wz = z > 0.f ? wi * rcp_approx(z) : 0.f;  // A_in = O / z
+      const float* crow = ca_s + r * kCS;
+      __nv_bfloat16* dst = p.a_full + fe * D;
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        const int col = n * 8 + 2 * (lane & 3);
+        const float2 ao = *reinterpret_cast<const float2*>(crow + col);
+        *reinterpret_cast<__nv_bfloat162*>(dst + col) = __floats2bfloat162_rn(
+            fmaf(wo, ao.x, wz * acc.o[n][2 * i]), fmaf(wo, ao.y, wz * acc.o[n][2 * i + 1]));
+      }
+      if ((lane & 3) == 0 && p.l_full) p.l_full[fe] = lf2 == kNegInf ? kNegInf : lf2 * kLn2;
+    }
+  }
+}
+
+// The rows of a served group that CTA `split` of its S takes: whole 16-row warp
+// slabs, dealt out as evenly as the slabs allow.
+__device__ __forceinline__ void lean_rows(int nrows, int split, int S, int& r0, int& nr) {
+  const int slabs = (nrows + 15) / 16;
+  const int per = (slabs + S - 1) / S;
+  r0 = min(nrows, split * per * 16);
+  nr = min(nrows, (split + 1) * per * 16) - r0;
+}
+
+}  // namespace fb

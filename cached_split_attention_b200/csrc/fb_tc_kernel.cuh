@@ -187,8 +187,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   const bool merger = cluster_mode || has_in || (S == 1 && has_out);
 
   if (p.decision_out && t == 0 && split == S - 1 && tid < g) p.decision_out[b * p.hq + hk * g + tid] = s_rec[tid];
-
-  if (active && (has_in || has_out || cluster_mode)) {
+  // A group whose heads all reuse takes the lean reuse path (its CTAs share the rows).
+  const bool lean = p.lean && !any_rec && active;
+  if (lean) {
+    int r0, nr;
+    lean_rows(nrows, split, S, r0, nr);
+    if (n_in > p.reuse_chunks * kBN) {
+      if (tid == 0) record_status(kDevBadIndex);
+    } else if (nr > 0) {
+      lean_reuse<kD>(p, smem, b, hk, q0, in0, n_in, row0 + r0, nr, tid, kThreads);
+    }
+  } else if (active && (has_in || has_out || cluster_mode)) {
     // -------------------------------------------------------- Q rows (before the K/V stream)
     constexpr int kQVec = kM * (kD / 8);
     constexpr int kQPer = (kQVec + kThreads - 1) / kThreads;

@@ -315,10 +315,13 @@ def video(seed: int = 1004, steps: int = 10, block: int = 1560, prefix_blocks: i
     """Video-shaped: batch 1, H=40, d=128, block 1560 query tokens, prefix 6 blocks
     (9360 tokens), 10 steps, per-head cosine gate gamma=0.95, tau gate off.
 
-    Prefix and initial block Q, K, V ~ N(0,1).  Each step adds sigma_h * N(0,1),
-    cumulatively, to the block Q/K/V of head h (float32 state, rounded to bf16
-    after each step); a seeded random half of the heads gets sigma=0.02, the other
-    half sigma=0.5."""
+    Prefix and initial block Q, K, V ~ N(0,1).  Each step perturbs the block Q/K/V
+    of head h with step noise sigma_h in variance-preserving form,
+    x <- (x + sigma_h * N(0,1)) / sqrt(1 + sigma_h^2) (float32 state, rounded to
+    bf16 after each step), so the activations keep their N(0,1) scale from step to
+    step (a denoising step does not inflate them) while consecutive steps of a head
+    have cosine about 1 / sqrt(1 + sigma_h^2); a seeded random half of the heads
+    gets sigma=0.02 (cosine 0.9998 per step), the other half sigma=0.5 (0.894)."""
     rng = np.random.default_rng(seed)
     N = prefix_blocks * block
     p = make_problem([np.arange(block)], [N], [block], heads, heads, head_dim)
@@ -335,13 +338,16 @@ def video(seed: int = 1004, steps: int = 10, block: int = 1560, prefix_blocks: i
         return StepInput(q=f32_to_bf16_bits(q), k_in=f32_to_bf16_bits(k), v_in=f32_to_bf16_bits(v),
                          n_updated=np.array([block], np.int32), problem=p)
 
+    keep = (1.0 / np.sqrt(1.0 + sigma.astype(np.float64) ** 2)).astype(np.float32)
     out = [snap()]
     for _ in range(1, steps):
         for x in (q, k, v):
             x += sigma[None, :, None] * rng.standard_normal(x.shape, dtype=np.float32)
+            x *= keep[None, :, None]
         out.append(snap())
     w = Workload("video", p, k_out, v_out, out, tau=0, gamma=gamma, flags=GATE_HEAD,
-                 notes="H40 d128 block1560 prefix9360; cumulative noise sigma 0.02/0.5 on halves; gamma=0.95")
+                 notes="H40 d128 block1560 prefix9360; variance-preserving step noise sigma 0.02/0.5 on halves; "
+                       "gamma=0.95")
     w.sigma = sigma  # type: ignore[attr-defined]
     return w
 
@@ -376,6 +382,35 @@ def locking_tiny(seed: int = 1010, steps: int = 5, block: int = 48, prefix: int 
         out.append(st.step_input([len(t) for t in toks], p))
     return Workload("locking_tiny", p0, k_out, v_out, out, tau=4, gamma=0.0, flags=GATE_TAU,
                     notes="2 seqs, GQA 4/2, d64, monotone locking, 3 redraws/step")
+
+
+def next_block(w: Workload, seed: int, steps: int = 4, redraws: int = 2, name: str = "") -> Workload:
+    """Inputs of the block that follows ``w``'s: same block lengths and the same
+    active block positions as ``w``'s first step, each sequence's prefix longer by
+    its finished block (J_out grows by B_b tokens), fresh Q/K/V for the new block,
+    and ``redraws`` updated tokens per sequence and step (tau gate as in ``w``).
+
+    Shapes and draws only: k_out / v_out are left as None -- the grown prefix (the
+    old prefix followed by the finished block's K/V) is made by the block
+    transition itself."""
+    rng = np.random.default_rng(seed)
+    p1 = w.steps[0].problem
+    lens_out = p1.lens("out") + p1.lens("in")
+    rows = [p1.q_rows[p1.cu_seqlens_q[b]:p1.cu_seqlens_q[b + 1]] for b in range(p1.num_seqs)]
+    p = make_problem(rows, lens_out, p1.lens("in"), p1.num_heads_q, p1.num_heads_kv, p1.head_dim,
+                     p1.softmax_scale)
+    st = _BlockState(rng, p, 1.0, 1.0)
+    out = [st.step_input(p.lens("in"))]
+    for _ in range(1, steps):
+        toks = []
+        for b, r in enumerate(rows):
+            k = min(redraws, len(r))
+            if k:
+                toks.append(np.sort(rng.choice(r, size=k, replace=False)) + p.cu_seqlens_kv_in[b])
+        st.redraw(np.concatenate(toks) if toks else np.zeros(0, np.int64))
+        out.append(st.step_input([min(redraws, len(r)) for r in rows]))
+    return Workload(name or w.name + "_next_block", p, None, None, out, tau=w.tau, gamma=w.gamma, flags=w.flags,
+                    notes="the block after " + w.name)
 
 
 def first_sequences(w: Workload, n: int) -> Workload:

@@ -157,6 +157,12 @@ typedef struct fb_plan_info {
   int32_t smem_bytes;     /* dynamic shared memory per CTA                          */
   int32_t keys_per_chunk; /* keys per pipeline stage (TMA box rows)                 */
   int32_t num_sms;        /* SM count the plan was made for                         */
+  /* Lean reuse path of fb_step (blocks of at most 128 keys): a work item whose
+   * q-heads all reuse the cache skips the streaming pipeline; its CTAs share its
+   * rows and run the block attention and the merge with the cached partial from
+   * one round of loads. */
+  int32_t lean_reuse;      /* 1 when the call has the lean path                     */
+  int32_t lean_smem_bytes; /* shared memory it uses per CTA at most (of smem_bytes) */
 } fb_plan_info;
 
 /*
@@ -292,6 +298,29 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
                            int32_t total_sel, const fb_bf16* k_out, const fb_bf16* v_out, const fb_bf16* k_in,
                            const fb_bf16* v_in, fb_bf16* k_res, fb_bf16* v_res, fb_bf16* k_ext, fb_bf16* v_ext,
                            int32_t* cu_seqlens_kv_out_res, int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream);
+
+/*
+ * Block transition (FlashBlock, gist.science/es/paper/2602.05305, "Mecanismo Central": a
+ * finished block stops being denoised and its tokens become context of the next block,
+ * i.e. part of its out-of-block set J_out).  For every sequence b:
+ *   J_out'(b) = J_out(b) followed by J_in(b) (block order),  cu_out'[b] = cu_out[b] + cu_in[b]
+ * k_out, v_out [total_kv_out, H_kv, d] and k_in, v_in [total_kv_in, H_kv, d] (THD bf16,
+ * device) are the prefix and the finished block's final K/V; the result goes to k_dst,
+ * v_dst [total_kv_out + total_kv_in, H_kv, d] (device, caller-owned) and, when not NULL,
+ * cu_seqlens_kv_out_dst [num_seqs+1] (device).
+ *   - New buffers (k_dst != k_out): every prefix row and block row is copied; the source
+ *     and destination must not overlap.
+ *   - In place (k_dst == k_out and v_dst == v_out; one sequence only, the buffers must
+ *     hold total_kv_out + total_kv_in rows): only the block rows are written, after the
+ *     prefix.  FB_ERR_UNSUPPORTED for more sequences (later ones would have to move).
+ * The next block brings new queries: call fb_cache_invalidate before its first fb_step
+ * (every head then recomputes over the grown prefix).  Asynchronous on `stream`; index
+ * arrays that disagree with the host totals record FB_ERR_INVALID_ARG on the device
+ * (that sequence is skipped).  At most 65535 sequences per call.
+ */
+fb_status fb_prefix_append(const fb_problem* problem, const fb_bf16* k_out, const fb_bf16* v_out,
+                           const fb_bf16* k_in, const fb_bf16* v_in, fb_bf16* k_dst, fb_bf16* v_dst,
+                           int32_t* cu_seqlens_kv_out_dst, fb_stream_t stream);
 
 /*
  * Self-test of the failure path of the bounded waits (no counterpart in the pages):

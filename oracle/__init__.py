@@ -19,6 +19,9 @@ Contents
                 policy that keeps the (A_out, L_out) cache.
   brute.py      pure-Python (math.fsum) restatement of the definition, used to pin
                 attention.py on tiny inputs.
+  transition.py the block transition: a finished block's K/V join each sequence's
+                prefix (FlashBlock, "Mecanismo Central": finished tokens become
+                out-of-block context) and the next block starts from an empty cache.
   sparse.py     the sparse-residual variant (FlashBlock, "Estrategias de Reutilizacion
                 Adaptativa", third bullet): keys a sparse pattern leaves out form the
                 cached out-of-block set; the selected ones join the block's keys.
@@ -31,4 +34,4 @@ reuse approximation error, which the oracle reports for information only.
 """
 from .attention import attend, attend_problem, bf16_to_f64, merge  # noqa: F401
 from .policy import OracleCache, decide, head_cosine, run_policy  # noqa: F401
-from . import sparse  # noqa: F401
+from . import sparse, transition  # noqa: F401

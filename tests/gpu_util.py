@@ -51,15 +51,17 @@ def workspace_for(steps_problems, out_splits=0, device="cuda"):
     return ws
 
 
-def run_policy_gpu(w, flags=None, out_splits=0, head_reuse_in=None, device="cuda", keep=True, cache=None):
+def run_policy_gpu(w, flags=None, out_splits=0, head_reuse_in=None, device="cuda", keep=True, cache=None,
+                   k_out=None, v_out=None):
     """Run a workload's steps through fb_step (on ``cache`` when given, else on a new
-    empty one); returns per-step dicts of numpy arrays and the cache."""
+    empty one; on the device prefix ``k_out``/``v_out`` when given, else on w's
+    uploaded); returns per-step dicts of numpy arrays and the cache."""
     torch, B = torch_and_binding()
     flags = w.flags if flags is None else flags
     p0 = w.problem
     cache = cache if cache is not None else B.Cache(p0, device, with_q_ref=True)
-    k_out = B.bf16_tensor(w.k_out, device)
-    v_out = B.bf16_tensor(w.v_out, device)
+    k_out = B.bf16_tensor(w.k_out, device) if k_out is None else k_out
+    v_out = B.bf16_tensor(w.v_out, device) if v_out is None else v_out
     ws = workspace_for([st.problem for st in w.steps], out_splits, device)
     prm = B.params(w.tau, w.gamma, flags)
     out = []

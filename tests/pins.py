@@ -350,6 +350,78 @@ def check_sparse_workload(sparse_workload, run_policy, attend_full):
             _close(r.l_full, l_ex, what=f"{w.name} sparse step {s} L")
 
 
+# ---------------------------------------------------------------- block transition
+
+def _transition_case():
+    """Block 1: two sequences (GQA 4/2, d = 16), prefixes 37 and 0, blocks 20 and 9
+    with a few locked rows, 3 steps that redraw tokens; block 2: the block after it."""
+    from cached_split_attention_b200 import workloads as W
+    rng = np.random.default_rng(11)
+    p = W.make_problem([[0, 2, 3, 7, 8, 11, 19], [0, 1, 4, 8]], [37, 0], [20, 9], 4, 2, 16)
+    k_out = W.normal_bf16(rng, (p.total_kv_out, 2, 16), 0.7)
+    v_out = W.normal_bf16(rng, (p.total_kv_out, 2, 16))
+    st = W._BlockState(rng, p, 0.7, 0.7, 1.0)
+    steps = [st.step_input([20, 9])]
+    for _ in range(2):
+        st.redraw(np.array([2, 11, 20 + 4]))
+        steps.append(st.step_input([2, 1]))
+    w1 = W.Workload("transition_case", p, k_out, v_out, steps, tau=2, gamma=0.0, flags=W.GATE_TAU)
+    return w1, W.next_block(w1, seed=12, steps=3, redraws=1)
+
+
+def check_block_transition(grow_prefix, finish_block, next_block_workload, run_policy, attend):
+    """Block transition (FlashBlock, "Mecanismo Central": the finished block's tokens
+    leave J_in and become context, i.e. J_out of the next block).
+    1. A hand-made case: prefixes of lengths 2 and 0, blocks of 1 and 2 tokens with
+       distinct values: J_out' = [p0 p1 b0] and [b1 b2], cu = [0, 3, 5].
+    2. The grown prefix is the finished block's *last* step K/V after each prefix.
+    3. The next block's first step (empty cache) equals attention of its queries over
+       the old prefix, the finished block's final K/V and the new block's K/V,
+       concatenated here by hand per sequence and head."""
+    from cached_split_attention_b200.workloads import make_problem
+    p = make_problem([[0], [0, 1]], [2, 0], [1, 2], 1, 1, 1)
+    ko = np.array([[[1]], [[2]]], dtype=np.uint16); vo = ko + 100
+    ki = np.array([[[10]], [[11]], [[12]]], dtype=np.uint16); vi = ki + 100
+    cu, k2, v2 = grow_prefix(p, ko, vo, ki, vi)
+    assert list(cu) == [0, 3, 5], cu
+    assert k2.reshape(-1).tolist() == [1, 2, 10, 11, 12], k2.reshape(-1)
+    assert v2.reshape(-1).tolist() == [101, 102, 110, 111, 112], v2.reshape(-1)
+
+    from oracle.attention import bf16_to_f64
+    w1, nxt = _transition_case()
+    cu, k2, v2 = finish_block(w1)
+    last = w1.steps[-1]
+    assert not np.array_equal(last.k_in, w1.steps[0].k_in), "the case must redraw"
+    pl = last.problem
+    for b in range(pl.num_seqs):
+        o0, o1 = int(pl.cu_seqlens_kv_out[b]), int(pl.cu_seqlens_kv_out[b + 1])
+        i0, i1 = int(pl.cu_seqlens_kv_in[b]), int(pl.cu_seqlens_kv_in[b + 1])
+        n0 = int(cu[b])
+        assert int(cu[b + 1]) - n0 == (o1 - o0) + (i1 - i0)
+        assert np.array_equal(k2[n0:n0 + o1 - o0], w1.k_out[o0:o1])
+        assert np.array_equal(k2[n0 + o1 - o0:int(cu[b + 1])], last.k_in[i0:i1])
+        assert np.array_equal(v2[n0 + o1 - o0:int(cu[b + 1])], last.v_in[i0:i1])
+    w2 = next_block_workload(w1, nxt)
+    r0 = run_policy(w2)[0]
+    st2 = w2.steps[0]
+    p2 = st2.problem
+    g = p2.num_heads_q // p2.num_heads_kv
+    q = bf16_to_f64(st2.q)
+    for b in range(p2.num_seqs):
+        r_0, r_1 = int(p2.cu_seqlens_q[b]), int(p2.cu_seqlens_q[b + 1])
+        o0, o1 = int(pl.cu_seqlens_kv_out[b]), int(pl.cu_seqlens_kv_out[b + 1])
+        i0, i1 = int(pl.cu_seqlens_kv_in[b]), int(pl.cu_seqlens_kv_in[b + 1])
+        j0, j1 = int(p2.cu_seqlens_kv_in[b]), int(p2.cu_seqlens_kv_in[b + 1])
+        for h in range(p2.num_heads_q):
+            hk = h // g
+            kk = np.concatenate([w1.k_out[o0:o1, hk], last.k_in[i0:i1, hk], st2.k_in[j0:j1, hk]])
+            vv = np.concatenate([w1.v_out[o0:o1, hk], last.v_in[i0:i1, hk], st2.v_in[j0:j1, hk]])
+            a, l = attend(q[r_0:r_1, h], bf16_to_f64(kk), bf16_to_f64(vv), p2.softmax_scale)
+            _close(r0.a_full[r_0:r_1, h], a, what=f"next block step 0 A (seq {b}, head {h})")
+            _close(r0.l_full[r_0:r_1, h], l, what=f"next block step 0 L (seq {b}, head {h})")
+    assert r0.recompute.all()
+
+
 # ---------------------------------------------------------------- branch hooks
 
 def check_branch_hooks(cache_copy_seq, cache_invalidate_seqs):

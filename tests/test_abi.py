@@ -105,6 +105,14 @@ def test_host_validation_without_gpu():
     many = _problem(B, num_seqs=70000, total_q=0, max_q=0, total_kv_in=0, max_kv_in=0, total_kv_out=0, max_kv_out=0)
     rc = B._lib.fb_sparse_layout(ctypes.byref(many), 16, 16, 0, 16, 16, 16, 16, 16, 16, 16, 16, None, None, None)
     assert rc == B.ERR_UNSUPPORTED and "65535" in B.last_error()
+    # block transition: in place only for one sequence, K and V alike
+    two = _problem(B, num_seqs=2)
+    rc = B._lib.fb_prefix_append(ctypes.byref(two), 16, 32, 48, 64, 16, 32, None, None)
+    assert rc == B.ERR_UNSUPPORTED and "in-place" in B.last_error()
+    rc = B._lib.fb_prefix_append(ctypes.byref(ok), 16, 32, 48, 64, 16, 80, None, None)
+    assert rc == B.ERR_INVALID_ARG and "both" in B.last_error()
+    rc = B._lib.fb_prefix_append(ctypes.byref(ok), 16, 32, 48, 64, None, 80, None, None)
+    assert rc == B.ERR_INVALID_ARG and "k_dst" in B.last_error()
 
 
 def test_workspace_size_is_counter_plus_scores():
@@ -170,6 +178,22 @@ def test_plan_query_matches_the_bench_kernel_map():
     assert (dllm["rows_per_tile"], dllm["tiles"], dllm["work_items"]) == (32, 1, 32)
     gqa = B.plan_query(B.DeviceProblem(_shape_problems()["long_context_gqa"], "cpu"))
     assert (gqa["rows_per_tile"], gqa["tiles"], gqa["work_items"]) == (128, 1, 64)
+
+
+def test_plan_query_lean_reuse_path():
+    """The lean reuse path: planned for fused steps of blocks of at most 128 keys
+    (every bench workload but the 1560-token video block), never for the unfused
+    passes, and only when the kernel's shared memory holds what it needs."""
+    _built()
+    from cached_split_attention_b200 import binding as B
+    for name, p in _shape_problems().items():
+        dp = B.DeviceProblem(p, "cpu")
+        step = B.plan_query(dp, B.CALL_STEP)
+        assert step["lean_reuse"] == (0 if name == "video" else 1), (name, step)
+        if step["lean_reuse"]:
+            assert 0 < step["lean_smem_bytes"] <= step["smem_bytes"], (name, step)
+        for call in (B.CALL_OUT, B.CALL_IN):
+            assert B.plan_query(dp, call)["lean_reuse"] == 0
 
 
 def test_plan_query_rejects_bad_arguments():

@@ -149,7 +149,9 @@ def test_unmutated_oracle_passes_every_pin():
     pins.check_branch_hooks(policy.cache_copy_seq, policy.cache_invalidate_seqs)
     pins.check_policy_replay(policy.run_policy)
     pins.check_bf16_widening(attention.bf16_to_f64)
-    from oracle import sparse
+    from oracle import sparse, transition
+    pins.check_block_transition(transition.grow_prefix, transition.finish_block, transition.next_block_workload,
+                                policy.run_policy, attention.attend)
     pins.check_sparse_workload(sparse.sparse_workload, policy.run_policy, attention.attend_full)
 
 
@@ -249,3 +251,39 @@ def test_sparse_workload_mutants_caught(label, old, new):
     from oracle import sparse
     bad = mutate(sparse, "sparse_workload", old, new)
     assert caught(pins.check_sparse_workload, bad, policy.run_policy, attention.attend_full), label
+
+
+GROW_MUTANTS = [
+    ("block placed before the prefix", "ks.append(np.concatenate([k_out[o0:o1], k_in[i0:i1]]))",
+     "ks.append(np.concatenate([k_in[i0:i1], k_out[o0:o1]]))"),
+    ("values of the block taken from its keys", "vs.append(np.concatenate([v_out[o0:o1], v_in[i0:i1]]))",
+     "vs.append(np.concatenate([v_out[o0:o1], k_in[i0:i1]]))"),
+    ("block lengths left out of the new offsets", "lens.append((o1 - o0) + (i1 - i0))", "lens.append(o1 - o0)"),
+    ("blocks of the next sequence", "i0, i1 = int(cu_i[b]), int(cu_i[b + 1])",
+     "i0, i1 = int(cu_i[(b + 1) % problem.num_seqs]), int(cu_i[(b + 1) % problem.num_seqs + 1])"),
+]
+
+FINISH_MUTANTS = [
+    ("the block's first step instead of its last", "last = workload.steps[-1]", "last = workload.steps[0]"),
+]
+
+
+@pytest.mark.parametrize("label,old,new", GROW_MUTANTS, ids=[m[0] for m in GROW_MUTANTS])
+def test_grow_prefix_mutants_caught(label, old, new):
+    from oracle import transition
+    bad = mutate(transition, "grow_prefix", old, new)
+    bad_finish = mutate(transition, "finish_block", "last = workload.steps[-1]", "last = workload.steps[-1]",
+                        extra={"grow_prefix": bad})
+    bad_next = mutate(transition, "next_block_workload", "cu, k, v = finish_block(finished)",
+                      "cu, k, v = finish_block(finished)", extra={"finish_block": bad_finish})
+    assert caught(pins.check_block_transition, bad, bad_finish, bad_next, policy.run_policy, attention.attend), label
+
+
+@pytest.mark.parametrize("label,old,new", FINISH_MUTANTS, ids=[m[0] for m in FINISH_MUTANTS])
+def test_finish_block_mutants_caught(label, old, new):
+    from oracle import transition
+    bad = mutate(transition, "finish_block", old, new)
+    bad_next = mutate(transition, "next_block_workload", "cu, k, v = finish_block(finished)",
+                      "cu, k, v = finish_block(finished)", extra={"finish_block": bad})
+    assert caught(pins.check_block_transition, transition.grow_prefix, bad, bad_next, policy.run_policy,
+                  attention.attend), label

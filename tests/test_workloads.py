@@ -63,6 +63,23 @@ def test_video_sigma_halves():
     assert (w.sigma < 0.1).sum() == 4 and w.flags == W.GATE_HEAD
 
 
+def test_video_step_noise_keeps_the_scale():
+    """The step noise is variance-preserving: after 9 steps the block Q/K/V of every
+    head still have unit variance (a cumulative walk would reach 1 + 9 sigma^2 =
+    3.25 for sigma = 0.5), and a sigma = 0.5 head's queries at consecutive steps
+    have cosine close to 1 / sqrt(1 + 0.25) = 0.894."""
+    from oracle.attention import bf16_to_f64
+    w = W.video(steps=10, block=256, prefix_blocks=1, heads=8)
+    q0, q9 = bf16_to_f64(w.steps[0].q), bf16_to_f64(w.steps[9].q)
+    for x in (q9, bf16_to_f64(w.steps[9].k_in), bf16_to_f64(w.steps[9].v_in)):
+        var = x.var(axis=(0, 2))
+        assert np.all(np.abs(var - 1.0) < 0.05), var
+    hi = np.flatnonzero(w.sigma > 0.1)[0]
+    a, b = bf16_to_f64(w.steps[1].q)[:, hi].ravel(), q0[:, hi].ravel()
+    cos = a @ b / np.sqrt((a @ a) * (b @ b))
+    assert abs(cos - 1 / np.sqrt(1.25)) < 0.01, cos
+
+
 def test_dllm_default_recompute_steps():
     """The 8B-dLLM layer as the bench runs it (seed 1001): with tau = 4 the steps
     that recompute are 0, 2, 7, 12 and 25 (k = clamp(Poisson(2), 1, 4) reaches 4
