@@ -619,10 +619,12 @@ def sparse_selection(prefix_lens, seed: int = 7, sink: int = 64, window: int = 2
 
 
 def sparse_layout_bytes(p, total_sel: int) -> int:
-    """Bytes fb_sparse_layout must move: every prefix and block K/V row read once and
-    written once (to the residual prefix or the extended block), plus the indices."""
+    """Bytes fb_sparse_layout must move: the block rows and the selected prefix rows
+    (K and V) read once and written once into J_in', the prefix skip mask written, and
+    the index arrays read."""
     row = p.num_heads_kv * p.head_dim * 2 * 2          # K and V, bf16
-    return 2 * (p.total_kv_out + p.total_kv_in) * row + 4 * (total_sel + 3 * (p.num_seqs + 1))
+    mask = 4 * ((p.total_kv_out + 31) // 32)
+    return 2 * (p.total_kv_in + total_sel) * row + mask + 4 * (total_sel + 3 * (p.num_seqs + 1))
 
 
 def cache_copy_bytes(p, src: int, dst: int, with_q_ref: bool) -> int:
@@ -684,8 +686,8 @@ class _Single:
     """One layer of one step of a problem on the device: inputs, cache, workspace,
     outputs (the shapes fb_step wants)."""
 
-    def __init__(self, B, torch, problem, st, k_out, v_out, device, with_q_ref=False):
-        self.B, self.dp = B, B.DeviceProblem(problem, device)
+    def __init__(self, B, torch, problem, st, k_out, v_out, device, with_q_ref=False, kv_out_skip=None):
+        self.B, self.dp = B, B.DeviceProblem(problem, device, kv_out_skip=kv_out_skip)
         H, d = problem.num_heads_q, problem.head_dim
         self.q = B.bf16_tensor(st.q, device)
         self.k_in, self.v_in = B.bf16_tensor(st.k_in, device), B.bf16_tensor(st.v_in, device)
@@ -844,23 +846,21 @@ def _rows_sparse(torch, B, device, flush, flush_out, reps, clocks, out_rows, hbm
     Hk, d = p.num_heads_kv, p.head_dim
     k_out, v_out = B.bf16_tensor(w.k_out, device), B.bf16_tensor(w.v_out, device)
     dense = _Single(B, torch, p, st, k_out, v_out, device)
-    k_res = torch.empty((p.total_kv_out - total_sel, Hk, d), dtype=torch.bfloat16, device=device)
-    v_res = torch.empty_like(k_res)
     k_ext = torch.empty((p.total_kv_in + total_sel, Hk, d), dtype=torch.bfloat16, device=device)
     v_ext = torch.empty_like(k_ext)
-    cu_o = torch.empty(p.num_seqs + 1, dtype=torch.int32, device=device)
+    skip = torch.empty((p.total_kv_out + 31) // 32, dtype=torch.int32, device=device)
     cu_i = torch.empty(p.num_seqs + 1, dtype=torch.int32, device=device)
     d_cu_sel = torch.as_tensor(cu_sel).to(device)
     d_sel = torch.as_tensor(np.concatenate(sel)).to(device)
 
     def layout(stream_):
-        B.sparse_layout(dense.dp, d_cu_sel, d_sel, total_sel, k_out, v_out, dense.k_in, dense.v_in, k_res, v_res,
-                        k_ext, v_ext, cu_o, cu_i, stream=stream_)
+        B.sparse_layout(dense.dp, d_cu_sel, d_sel, total_sel, k_out, v_out, dense.k_in, dense.v_in, k_ext, v_ext,
+                        skip, cu_i, stream=stream_)
 
     g_lay = _graph_of(torch, layout)
     t_lay = _cold_us(torch, g_lay, flush, flush_out, reps, clocks)
-    p2 = dataclasses.replace(p, cu_seqlens_kv_out=cu_o.cpu().numpy(), cu_seqlens_kv_in=cu_i.cpu().numpy())
-    sp = _Single(B, torch, p2, dataclasses.replace(st, problem=p2), k_res, v_res, device)
+    p2 = dataclasses.replace(p, cu_seqlens_kv_in=cu_i.cpu().numpy())
+    sp = _Single(B, torch, p2, dataclasses.replace(st, problem=p2), k_out, v_out, device, kv_out_skip=skip)
     sp.k_in, sp.v_in = k_ext, v_ext
     timed = {}
     for name, obj in (("sparse", sp), ("dense", dense)):
@@ -877,6 +877,8 @@ def _rows_sparse(torch, B, device, flush, flush_out, reps, clocks, out_rows, hbm
     def arm(name, a, f):
         t = timed[(name, a)]
         b = step_bytes(p2 if name == "sparse" else p, f)["total"]
+        if name == "sparse":   # the selected keys are not streamed with the prefix
+            b -= f * total_sel * Hk * d * 2 * 2
         return dict(_stats(t), algorithmic_bytes=round(b), frac_of_hbm=round(b / float(np.median(t)) / 1e3 /
                                                                              hbm_peak, 4))
 

@@ -41,6 +41,7 @@ class FbProblem(ctypes.Structure):
         ("total_q", ctypes.c_int32), ("total_kv_out", ctypes.c_int32), ("total_kv_in", ctypes.c_int32),
         ("max_q", ctypes.c_int32), ("max_kv_out", ctypes.c_int32), ("max_kv_in", ctypes.c_int32),
         ("out_splits", ctypes.c_int32),
+        ("kv_out_skip", ctypes.c_void_p),
     ]
 
 
@@ -80,7 +81,7 @@ def _load():
         "fb_cache_invalidate": (st, [P, ctypes.POINTER(FbCache), vp]),
         "fb_cache_copy_seq": (st, [P, ctypes.POINTER(FbCache), ctypes.c_int32, ctypes.c_int32, vp]),
         "fb_cache_invalidate_seqs": (st, [P, ctypes.POINTER(FbCache), vp, vp]),
-        "fb_sparse_layout": (st, [P, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+        "fb_sparse_layout": (st, [P, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "fb_prefix_append": (st, [P, vp, vp, vp, vp, vp, vp, vp, vp]),
         "fb_selftest_wait_timeout": (st, [vp]),
         "fb_release_cache": (st, []),
@@ -133,9 +134,12 @@ def _stream(stream) -> Optional[int]:
 class DeviceProblem:
     """A problem with its index arrays uploaded to the device (int32)."""
 
-    def __init__(self, problem, device="cuda", out_splits: int = 0):
+    def __init__(self, problem, device="cuda", out_splits: int = 0, kv_out_skip=None):
+        """``kv_out_skip``: optional device uint32 bitmask over the prefix tokens (see
+        fb_problem in flashblock.h); it is kept alive with the problem."""
         import torch
         self.host = problem
+        self.kv_out_skip = kv_out_skip
         mk = lambda a: torch.as_tensor(np.ascontiguousarray(a, dtype=np.int32)).to(device)
         self.cu_q = mk(problem.cu_seqlens_q)
         self.q_rows = mk(problem.q_rows) if len(problem.q_rows) else None
@@ -145,7 +149,7 @@ class DeviceProblem:
             problem.num_seqs, problem.num_heads_q, problem.num_heads_kv, problem.head_dim,
             float(problem.softmax_scale), _ptr(self.cu_q), _ptr(self.q_rows), _ptr(self.cu_out), _ptr(self.cu_in),
             problem.total_q, problem.total_kv_out, problem.total_kv_in,
-            problem.max_q, problem.max_kv_out, problem.max_kv_in, int(out_splits))
+            problem.max_q, problem.max_kv_out, problem.max_kv_in, int(out_splits), _ptr(kv_out_skip))
 
     @property
     def ref(self):
@@ -256,12 +260,12 @@ def cache_invalidate_seqs(problem: DeviceProblem, cache: Cache, seq_mask=None, s
 
 
 def sparse_layout(problem: DeviceProblem, cu_sel, sel_idx, total_sel: int, k_out, v_out, k_in, v_in,
-                  k_res, v_res, k_ext, v_ext, cu_out_res=None, cu_in_ext=None, stream=None):
-    """fb_sparse_layout: selected prefix keys join the block's keys, the rest form the
-    residual prefix (see flashblock.h)."""
+                  k_ext, v_ext, kv_out_skip, cu_in_ext=None, stream=None):
+    """fb_sparse_layout: selected prefix keys join the block's keys (k_ext, v_ext) and are
+    marked in the prefix skip mask (see flashblock.h)."""
     _check(_lib.fb_sparse_layout(problem.ref, _ptr(cu_sel), _ptr(sel_idx), int(total_sel), _ptr(k_out), _ptr(v_out),
-                                 _ptr(k_in), _ptr(v_in), _ptr(k_res), _ptr(v_res), _ptr(k_ext), _ptr(v_ext),
-                                 _ptr(cu_out_res), _ptr(cu_in_ext), _stream(stream)))
+                                 _ptr(k_in), _ptr(v_in), _ptr(k_ext), _ptr(v_ext), _ptr(kv_out_skip),
+                                 _ptr(cu_in_ext), _stream(stream)))
 
 
 def prefix_append(problem: DeviceProblem, k_out, v_out, k_in, v_in, k_dst, v_dst, cu_out_dst=None, stream=None):

@@ -72,6 +72,8 @@ fb_status check_problem(const fb_problem* p) {
     return fail(FB_ERR_UNSUPPORTED, "num_seqs x num_heads_q x max_q is too large for one launch");
   if (p->num_seqs > 0 && (!p->cu_seqlens_q || !p->cu_seqlens_kv_out || !p->cu_seqlens_kv_in))
     return fail(FB_ERR_INVALID_ARG, "cu_seqlens arrays must not be NULL");
+  if (p->kv_out_skip && (reinterpret_cast<uintptr_t>(p->kv_out_skip) & 3u))
+    return fail(FB_ERR_INVALID_ARG, "kv_out_skip is not 4-byte aligned");
   return FB_OK;
 }
 
@@ -187,10 +189,21 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = fals
     if (p->out_splits > 0) {
       splits = p->out_splits;
     } else {
-      // One wave: as many CTAs per group as the resident slots allow.
+      // The split with the shortest makespan: S CTAs per group take ceil(G S /
+      // slots) waves of 1/S of a group's keys each, and every further split adds
+      // about 3 % for its partial's merge.  One wave when G <= slots: S = slots / G.
       const int per_sm = std::max(1, std::min(233472 / (pl.smem + 1024), 2048 / pl.threads));
       const long slots = static_cast<long>(num_sms) * per_sm;
-      splits = static_cast<int>(std::max(1L, slots / std::max(1, pl.n_groups)));
+      const long G = std::max(1, pl.n_groups);
+      double best = 1e30;
+      for (int s = 1; s <= fb::kMaxSplits; ++s) {
+        const double waves = static_cast<double>((G * s + slots - 1) / slots);
+        const double span = waves / s * (1.0 + 0.03 * (s - 1));
+        if (span < best - 1e-9) {
+          best = span;
+          splits = s;
+        }
+      }
     }
     splits = std::max(1, std::min({splits, fb::kMaxSplits, chunks}));
   }
@@ -354,6 +367,7 @@ void fill_problem(const fb_problem* p, const Plan& pl, fb::Params& prm) {
   prm.total_in = p->total_kv_in;
   prm.tiles = pl.tiles;
   prm.splits = pl.splits;
+  prm.out_skip = p->kv_out_skip;
 }
 
 void fill_workspace(const Plan& pl, void* ws, fb::Params& prm) {
@@ -564,9 +578,9 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   prm.a_full = reinterpret_cast<__nv_bfloat16*>(a_full);
   prm.l_full = l_full;
   prm.decision_out = decision_out;
-  if (pl.reuse) {
-    prm.k_in = reinterpret_cast<const __nv_bfloat16*>(k_in);
-    prm.v_in = reinterpret_cast<const __nv_bfloat16*>(v_in);
+  if (pl.reuse) {  // block K/V with 64-row boxes for the lean reuse path
+    FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, fb::kBN, &prm.tm_k_lean));
+    FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, fb::kBN, &prm.tm_v_lean));
     prm.reuse_chunks = pl.reuse_chunks;
     prm.lean = 1;
   }
@@ -629,8 +643,8 @@ fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* ca
 
 fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, const int32_t* sel_idx,
                            int32_t total_sel, const fb_bf16* k_out, const fb_bf16* v_out, const fb_bf16* k_in,
-                           const fb_bf16* v_in, fb_bf16* k_res, fb_bf16* v_res, fb_bf16* k_ext, fb_bf16* v_ext,
-                           int32_t* cu_seqlens_kv_out_res, int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream) {
+                           const fb_bf16* v_in, fb_bf16* k_ext, fb_bf16* v_ext, uint32_t* kv_out_skip,
+                           int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream) {
   FB_TRY(check_problem(problem));
   if (total_sel < 0 || total_sel > problem->total_kv_out)
     return fail(FB_ERR_INVALID_ARG, "total_sel %d outside [0, total_kv_out]", total_sel);
@@ -639,30 +653,36 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
     return fail(FB_ERR_UNSUPPORTED, "fb_sparse_layout takes at most 65535 sequences per call");
   if (!cu_sel) return fail(FB_ERR_INVALID_ARG, "cu_sel is NULL");
   if (total_sel > 0 && !sel_idx) return fail(FB_ERR_INVALID_ARG, "sel_idx is NULL");
-  const bool res = problem->total_kv_out - total_sel > 0;
   const bool ext = problem->total_kv_in + total_sel > 0;
   FB_TRY(check_ptr(k_out, "k_out", problem->total_kv_out > 0));
   FB_TRY(check_ptr(v_out, "v_out", problem->total_kv_out > 0));
   FB_TRY(check_ptr(k_in, "k_in", problem->total_kv_in > 0));
   FB_TRY(check_ptr(v_in, "v_in", problem->total_kv_in > 0));
-  FB_TRY(check_ptr(k_res, "k_res", res));
-  FB_TRY(check_ptr(v_res, "v_res", res));
   FB_TRY(check_ptr(k_ext, "k_ext", ext));
   FB_TRY(check_ptr(v_ext, "v_ext", ext));
+  if (problem->total_kv_out > 0 && !kv_out_skip) return fail(FB_ERR_INVALID_ARG, "kv_out_skip is NULL");
+  if (kv_out_skip && (reinterpret_cast<uintptr_t>(kv_out_skip) & 3u))
+    return fail(FB_ERR_INVALID_ARG, "kv_out_skip is not 4-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t words = (static_cast<size_t>(problem->total_kv_out) + 31) / 32;
+  if (words) {
+    cudaError_t e = cudaMemsetAsync(kv_out_skip, 0, words * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(kv_out_skip)");
+  }
   fb::SparseParams sp{problem->num_seqs, problem->num_heads_kv, problem->head_dim, problem->total_kv_out,
                       problem->total_kv_in, total_sel, problem->cu_seqlens_kv_out, problem->cu_seqlens_kv_in, cu_sel,
                       sel_idx, reinterpret_cast<const __nv_bfloat16*>(k_out),
                       reinterpret_cast<const __nv_bfloat16*>(v_out), reinterpret_cast<const __nv_bfloat16*>(k_in),
-                      reinterpret_cast<const __nv_bfloat16*>(v_in), reinterpret_cast<__nv_bfloat16*>(k_res),
-                      reinterpret_cast<__nv_bfloat16*>(v_res), reinterpret_cast<__nv_bfloat16*>(k_ext),
-                      reinterpret_cast<__nv_bfloat16*>(v_ext), cu_seqlens_kv_out_res, cu_seqlens_kv_in_ext};
-  const long per_seq = static_cast<long>(problem->max_kv_out + problem->max_kv_in) * problem->num_heads_kv *
-                       problem->head_dim / 8;
+                      reinterpret_cast<const __nv_bfloat16*>(v_in), reinterpret_cast<__nv_bfloat16*>(k_ext),
+                      reinterpret_cast<__nv_bfloat16*>(v_ext), kv_out_skip, cu_seqlens_kv_in_ext};
+  // rows of J_in' per sequence: the block plus the selection (at most the prefix)
+  const long per_seq = static_cast<long>(problem->max_kv_in + std::min(problem->max_kv_out, total_sel)) *
+                       problem->num_heads_kv * problem->head_dim / 8;
   const int bx = static_cast<int>(std::max<long>(1, std::min<long>((per_seq + 255) / 256, 256)));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(bx, problem->num_seqs);
   cfg.blockDim = dim3(256);
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;

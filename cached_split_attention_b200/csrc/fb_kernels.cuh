@@ -50,6 +50,17 @@ __device__ int g_status;  // first error recorded by any kernel (0 = none)
 
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// Bits [t0, t0 + 64) of a prefix-token bitmask (bit t % 32 of word t / 32) as one
+// 64-bit word, bit k = token t0 + k; words past the end (total_out tokens) read 0.
+__device__ __forceinline__ uint64_t skip_bits64(const uint32_t* bits, int total_out, int t0) {
+  const int nwords = (total_out + 31) >> 5;
+  const int w = t0 >> 5;
+  const int sh = t0 & 31;
+  auto word = [&](int i) -> uint64_t { return i < nwords ? static_cast<uint64_t>(__ldg(bits + i)) : 0ull; };
+  const uint64_t lo = word(w) | (word(w + 1) << 32);
+  return sh ? (lo >> sh) | (word(w + 2) << (64 - sh)) : lo;
+}
+
 struct alignas(64) Params {
   CUtensorMap tm_k_out, tm_v_out, tm_k_in, tm_v_in;
   // problem
@@ -87,9 +98,9 @@ struct alignas(64) Params {
   // workspace
   int* grid_ctr;     // completion counter of the cache-state epilogue (zero between calls)
   const int* order;  // work order of the two-tile kernel (NULL: CTA i takes item i)
+  const uint32_t* out_skip;  // prefix tokens left out of J_out (bitmask; NULL: none)
   // lean reuse path (fb_reuse.cuh)
-  const __nv_bfloat16* k_in;  // block K/V, plain pointers
-  const __nv_bfloat16* v_in;
+  CUtensorMap tm_k_lean, tm_v_lean;  // block K/V with 64-row boxes (the warp-MMA stage layout)
   int reuse_chunks;  // 64-key chunks of the longest block
   int lean;          // 1: groups whose heads all reuse take the lean path
 };
@@ -298,7 +309,8 @@ struct Acc {
 // key row of the warp inside the stage tile.
 template <int D, int KW>
 __device__ __forceinline__ void consume_keys(Acc<D>& acc, const uint32_t (&qf)[D / 16][4], uint32_t kb, uint32_t vb,
-                                             int kr0, int key0, int k_end, float scale_log2, int lane) {
+                                             int kr0, int key0, int k_end, float scale_log2, int lane,
+                                             uint64_t skip = 0ull) {
   float s[KW / 8][4];
 #pragma unroll
   for (int n = 0; n < KW / 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
@@ -315,13 +327,15 @@ __device__ __forceinline__ void consume_keys(Acc<D>& acc, const uint32_t (&qf)[D
       mma_bf16_16816(s[2 * nb + 1], qf[kk], r[2], r[3]);
     }
   }
-  const bool need_mask = key0 + KW > k_end;
+  // keys past the segment's end, and keys the skip mask leaves out (bit k = key key0 + k)
+  const bool need_mask = key0 + KW > k_end || skip != 0ull;
 #pragma unroll
   for (int n = 0; n < KW / 8; ++n) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       float v = s[n][e] * scale_log2;
-      if (need_mask && key0 + n * 8 + 2 * (lane & 3) + (e & 1) >= k_end) v = kNegInf;
+      const int rel = n * 8 + 2 * (lane & 3) + (e & 1);
+      if (need_mask && (key0 + rel >= k_end || ((skip >> rel) & 1ull))) v = kNegInf;
       s[n][e] = v;
     }
   }
@@ -589,9 +603,19 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
     bool ok = true;
     int issued = min(STAGES, n_local);
 
+    // skip-mask bits of the warp's keys of a prefix chunk (loaded one chunk ahead)
+    auto skip_of = [&](int c) -> uint64_t {
+      if (!p.out_skip || c < nA || c >= n_local) return 0ull;
+      uint64_t w = skip_bits64(p.out_skip, p.total_out, out0 + (pa + c - nA) * kBN + wn * KW);
+      if (KW < 64) w &= (1ull << KW) - 1ull;
+      return w;
+    };
     // One segment of chunks [c0, c1) of the local sequence.
     auto run = [&](int c0, int c1) {
+      uint64_t skip_next = skip_of(c0);
       for (int c = c0; c < c1 && ok; ++c) {
+        const uint64_t skip = skip_next;
+        skip_next = skip_of(c + 1);
         const int st = c % STAGES;
         // every lane waits; the warp leaves together if the wait ran out
         if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (c / STAGES) & 1))) {
@@ -604,7 +628,7 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
           const int key0 = (seg_in ? c * kBN : (pa + c - nA) * kBN) + wn * KW;
           const uint32_t kb = smem_u32(stages + st * C::kStageBytes);
           consume_keys<D, KW>(acc, qf, kb, kb + C::kTileBytes, wn * KW, key0, seg_in ? n_in : n_out, p.scale_log2,
-                              lane);
+                              lane, skip);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);

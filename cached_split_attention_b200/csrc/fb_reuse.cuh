@@ -10,9 +10,11 @@
 // TMA pipeline, cluster and merge phases.  The group's CTAs share its rows (16 per
 // warp) and each runs:
 //
-//   loads      Q rows, the block K/V of the kv-head and q_rows, all issued together
-//              as 16-byte cp.async into shared memory; then the cached A_out /
-//              L_out rows at the rows' block positions;
+//   loads      by TMA, completed on one mbarrier: the block K/V of the kv-head as
+//              64-row tensor-map boxes (whole 64-key chunks; keys past the block
+//              are masked), each row's Q as a 1-D bulk copy, and -- as soon as the
+//              row's block position (q_rows) is back -- its cached A_out entry
+//              (1-D bulk) and L_out;
 //   attention  S = Q K^T and O = P V with mma.sync (bf16 in, fp32 accumulate),
 //              online softmax in base 2 (the streaming kernel's inner loop);
 //   merge      in registers: A_full = w_out A_out + w_in A_in, L_full =
@@ -20,7 +22,8 @@
 //
 // K and V sit in shared memory in the 128-byte swizzled layout of the warp-MMA
 // kernel's stages (64-key chunks), so the same inner loop serves both.  Keys past
-// the block's end are zero-filled and masked.  Blocks of up to kMaxKeys keys take
+// the block's end are masked (rows past the tensor's end arrive as zeros, rows of
+// the next sequence are finite).  Blocks of up to kMaxKeys keys take
 // this path (the host plan checks max_kv_in and the shared memory it needs);
 // longer blocks are real contractions and stay on the streaming pipelines.
 //
@@ -39,7 +42,8 @@ __host__ __device__ constexpr int tile_bytes(int d) { return kBN * d * 2; }
 __host__ __device__ constexpr int q_stride(int d) { return d + 8; }  // padded bf16 Q row
 __host__ __device__ constexpr int c_stride(int d) { return d + 4; }  // padded fp32 cache row
 __host__ __device__ constexpr int smem_bytes(int d, int chunks, int rows) {
-  return 2 * chunks * tile_bytes(d) + rows * q_stride(d) * 2 + rows * c_stride(d) * 4 + rows * 4 + rows * 4;
+  // K, V chunks; Q rows; cache A rows; cache L; output entry of each row; the barrier
+  return 2 * chunks * tile_bytes(d) + rows * q_stride(d) * 2 + rows * c_stride(d) * 4 + rows * 4 + rows * 4 + 16;
 }
 
 }  // namespace reuse
@@ -51,8 +55,6 @@ __host__ __device__ constexpr int smem_bytes(int d, int chunks, int rows) {
 template <int D>
 __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b, int hk, int q0, int in0, int n_in,
                                            int r0, int nr, int tid, int nthreads) {
-  constexpr int kVec = D / 8;   // 16-byte vectors of a bf16 row
-  constexpr int kCVec = D / 4;  // 16-byte vectors of an fp32 row
   constexpr int kT = reuse::tile_bytes(D);
   constexpr int kQS = reuse::q_stride(D);
   constexpr int kCS = reuse::c_stride(D);
@@ -64,68 +66,65 @@ __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b
   __nv_bfloat16* q_s = reinterpret_cast<__nv_bfloat16*>(smem + 2 * nch * kT);
   float* ca_s = reinterpret_cast<float*>(smem + 2 * nch * kT + nr16 * kQS * 2);
   float* cl_s = ca_s + nr16 * kCS;
-  int* pos_s = reinterpret_cast<int*>(cl_s + nr16);
+  int* fe_s = reinterpret_cast<int*>(cl_s + nr16);  // output entry of each row; -1: no output
+  uint64_t* bar = reinterpret_cast<uint64_t*>(fe_s + nr16);
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  const int used = (n_in + kBN - 1) / kBN;  // 64-key chunks holding the block
 
-  // Block K/V of kv-head hk: key rows up to the next multiple of 32 (the MMA's key
-  // slice); rows past the block's end are zero (masked scores, zero values).
-  const int n_keys = (n_in + 31) & ~31;
-  for (int it = tid; it < 2 * n_keys * kVec; it += nthreads) {
-    const int is_v = it >= n_keys * kVec;
-    const int v = is_v ? it - n_keys * kVec : it;
-    const int kr = v / kVec;
-    const int c = v % kVec;
-    uint8_t* dst = (is_v ? vs : ks) + (kr / kBN) * kT + swz(kr % kBN, c * 8);
-    if (kr < n_in) {
-      const __nv_bfloat16* src = (is_v ? p.v_in : p.k_in) + (static_cast<size_t>(in0 + kr) * p.hkv + hk) * D + c * 8;
-      cp_async_16(dst, src);
-    } else {
-      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
+  // One thread per row reads its block position (the cache entry depends on it);
+  // thread 0 arms the barrier: one arrival per row, one for the block K/V.
+  int pos = -1, fe = -1;
+  if (tid < nr) {
+    const int rho = r0 + tid;
+    const int tok = rho / g;
+    pos = p.q_rows ? p.q_rows[q0 + tok] : tok;
+    fe = (q0 + tok) * p.hq + hk * g + (rho - tok * g);
   }
-  for (int it = tid; it < nr16 * kVec; it += nthreads) {
-    const int r = it / kVec;
-    const int c = it % kVec;
-    __nv_bfloat16* dst = q_s + r * kQS + c * 8;
-    if (r < nr) {
-      const int rho = r0 + r;
-      cp_async_16(dst, p.q + (static_cast<size_t>(q0 + rho / g) * p.hq + hk * g + rho % g) * D + c * 8);
-    } else {
-      *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
+  if (tid == 0) {
+    mbar_init(bar, nr + 1);
+    fence_barrier_init();
   }
-  cp_async_commit();
-  for (int r = tid; r < nr16; r += nthreads) {
-    int pos = -1;
-    if (r < nr) {
-      const int rho = r0 + r;
-      pos = p.q_rows ? p.q_rows[q0 + rho / g] : rho / g;
-      if (pos < 0 || pos >= n_in) {
-        record_status(kDevBadIndex);
-        pos = -1;
+  __syncthreads();
+  if (tid == 0) {  // block K/V of kv-head hk, whole 64-key chunks (keys past the block are masked)
+    mbar_arrive_expect_tx(bar, 2 * used * kT);
+    for (int c = 0; c < used; ++c) {
+#pragma unroll
+      for (int hh = 0; hh < D / 64; ++hh) {
+        tma_load_2d_plain(ks + c * kT + hh * (kBN * 128), &p.tm_k_lean, bar, hk * D + hh * 64, in0 + c * kBN);
+        tma_load_2d_plain(vs + c * kT + hh * (kBN * 128), &p.tm_v_lean, bar, hk * D + hh * 64, in0 + c * kBN);
       }
     }
-    pos_s[r] = pos;
   }
-  __syncthreads();
-  // cached rows at the block positions
-  for (int it = tid; it < nr * (kCVec + 1); it += nthreads) {
-    const int r = it / (kCVec + 1);
-    const int c = it % (kCVec + 1);
-    const int pos = pos_s[r];
-    if (pos < 0) continue;
-    const size_t ce = static_cast<size_t>(in0 + pos) * p.hq + hk * g + (r0 + r) % g;
-    if (c < kCVec) {
-      cp_async_16(ca_s + r * kCS + c * 4, p.cache_a + ce * D + c * 4);
+  if (tid < nr) {  // the row's Q, then (once its position is back) its cache entry
+    mbar_expect_tx(bar, D * 2);
+    bulk_load_1d(q_s + tid * kQS, p.q + static_cast<size_t>(fe) * D, D * 2, bar);
+    if (pos < 0 || pos >= n_in) {
+      record_status(kDevBadIndex);
+      fe = -1;
+      mbar_arrive(bar);
     } else {
-      cp_async_4(cl_s + r, p.cache_l + ce);
+      const size_t ce = static_cast<size_t>(in0 + pos) * p.hq + (fe % p.hq);
+      mbar_arrive_expect_tx(bar, D * 4);
+      bulk_load_1d(ca_s + tid * kCS, p.cache_a + ce * D, D * 4, bar);
+      cl_s[tid] = p.cache_l[ce];
     }
+  } else if (tid < nr16) {
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4*>(q_s + tid * kQS + c * 8) = make_uint4(0u, 0u, 0u, 0u);
   }
-  cp_async_commit();
-  cp_async_wait_all();
+  if (tid < nr16) fe_s[tid] = fe;
+  // every thread waits for the copies; on a timeout (never expected) the copies
+  // still in flight get a second bounded wait before the CTA moves on
+  bool ok = mbar_wait(bar, 0);
+  if (!ok) {
+    if (tid == 0) record_status(kDevTimeout);
+    mbar_wait(bar, 0);
+  }
   __syncthreads();
+  if (!ok) return;
 
+  const int n_keys = (n_in + 31) & ~31;
   for (int slab = warp; slab * 16 < nr; slab += nthreads / 32) {
     uint32_t qf[D / 16][4];
 #pragma unroll
@@ -142,9 +141,8 @@ __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b
     for (int i = 0; i < 2; ++i) {
       const float z = quad_sum(acc.l[i]);
       const int r = 16 * slab + (lane >> 2) + 8 * i;
-      if (r >= nr || pos_s[r] < 0) continue;
-      const int rho = r0 + r;
-      const size_t fe = static_cast<size_t>(q0 + rho / g) * p.hq + hk * g + rho % g;
+      const int e = fe_s[r];
+      if (e < 0) continue;
       const float li2 = z > 0.f ? acc.m[i] + lg2_approx(z) : kNegInf;
       const float lo_nat = cl_s[r];
       const float lo2 = lo_nat == kNegInf ? kNegInf : lo_nat * kLog2e;
@@ -160,7 +158,7 @@ __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b
       }
       const float wz = z > 0.f ? wi * rcp_approx(z) : 0.f;  // A_in = O / z
       const float* crow = ca_s + r * kCS;
-      __nv_bfloat16* dst = p.a_full + fe * D;
+      __nv_bfloat16* dst = p.a_full + static_cast<size_t>(e) * D;
 #pragma unroll
       for (int n = 0; n < D / 8; ++n) {
         const int col = n * 8 + 2 * (lane & 3);
@@ -168,7 +166,7 @@ __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b
         *reinterpret_cast<__nv_bfloat162*>(dst + col) = __floats2bfloat162_rn(
             fmaf(wo, ao.x, wz * acc.o[n][2 * i]), fmaf(wo, ao.y, wz * acc.o[n][2 * i + 1]));
       }
-      if ((lane & 3) == 0 && p.l_full) p.l_full[fe] = lf2 == kNegInf ? kNegInf : lf2 * kLn2;
+      if ((lane & 3) == 0 && p.l_full) p.l_full[e] = lf2 == kNegInf ? kNegInf : lf2 * kLn2;
     }
   }
 }

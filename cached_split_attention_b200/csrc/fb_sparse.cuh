@@ -2,8 +2,11 @@
 // Adaptativa", third bullet: the keys a sparse pattern does not select form the
 // out-of-block set whose contribution is cached).  Per sequence b, the selected
 // prefix keys join the block's keys -- J_in' = block keys, then the selected keys
-// in increasing order -- and the others form the residual prefix J_out' (order
-// kept).  The attention kernels then run unchanged on (J_out', J_in').
+// in increasing order -- and the others form the residual prefix J_out'.  The
+// residual is not copied: the selected prefix tokens are marked in a bitmask that
+// the prefix pass of every attention kernel consults (fb_problem.kv_out_skip), so
+// this pass moves only the block rows and the selected rows (a few MB) instead of
+// the whole prefix.
 #pragma once
 
 #include "fb_device.cuh"
@@ -21,17 +24,15 @@ struct SparseParams {
   const __nv_bfloat16* v_out;
   const __nv_bfloat16* k_in;
   const __nv_bfloat16* v_in;
-  __nv_bfloat16* k_res;
-  __nv_bfloat16* v_res;
   __nv_bfloat16* k_ext;
   __nv_bfloat16* v_ext;
-  int* cu_out_res;  // optional: cu_out - cu_sel
+  uint32_t* skip;   // bit t: prefix token t selected (cleared by the host beforehand)
   int* cu_in_ext;   // optional: cu_in + cu_sel
 };
 
-// blockIdx.y = sequence; the x-blocks stride over (token, 16-byte piece) items of
-// the sequence's prefix then block rows.  Each prefix token finds its rank among
-// the selected positions by binary search.
+// blockIdx.y = sequence; the x-blocks stride over (row, 16-byte piece) items of the
+// sequence's J_in' rows: its block rows, then its selected prefix rows.  The first
+// x-block also sets the skip bits of the selected tokens.
 __global__ void __launch_bounds__(256) sparse_layout_kernel(const SparseParams p) {
   pdl_wait();
   pdl_trigger();
@@ -52,50 +53,28 @@ __global__ void __launch_bounds__(256) sparse_layout_kernel(const SparseParams p
     if (blockIdx.x == 0 && threadIdx.x == 0) record_status(kDevBadIndex);
     return;
   }
-  const int r0 = o0 - s0;  // J_out' of b starts here
   const int e0 = i0 + s0;  // J_in' of b starts here
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    if (p.cu_out_res) p.cu_out_res[b] = r0;
-    if (p.cu_in_ext) p.cu_in_ext[b] = e0;
-    if (b == p.num_seqs - 1) {
-      if (p.cu_out_res) p.cu_out_res[b + 1] = p.cu_out[b + 1] - p.cu_sel[b + 1];
-      if (p.cu_in_ext) p.cu_in_ext[b + 1] = p.cu_in[b + 1] + p.cu_sel[b + 1];
+  if (blockIdx.x == 0) {
+    if (threadIdx.x == 0 && p.cu_in_ext) {
+      p.cu_in_ext[b] = e0;
+      if (b == p.num_seqs - 1) p.cu_in_ext[b + 1] = p.cu_in[b + 1] + p.cu_sel[b + 1];
+    }
+    for (int k = threadIdx.x; k < n_sel; k += blockDim.x) {
+      const int t = o0 + p.sel[s0 + k];
+      atomicOr(p.skip + (t >> 5), 1u << (t & 31));
     }
   }
   const int vec = p.hkv * p.d / 8;  // 16-byte pieces per token row
-  const long items = static_cast<long>(n_out + n_in) * vec;
+  const long items = static_cast<long>(n_in + n_sel) * vec;
   for (long it = blockIdx.x * 256l + threadIdx.x; it < items; it += static_cast<long>(gridDim.x) * 256) {
-    const int tok = static_cast<int>(it / vec);
+    const int row = static_cast<int>(it / vec);
     const int c = static_cast<int>(it % vec) * 8;
-    const uint4* sk;
-    const uint4* sv;
-    uint4* dk;
-    uint4* dv;
-    if (tok < n_out) {
-      int lo = 0, hi = n_sel;  // rank = number of selected positions below tok
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (p.sel[s0 + mid] < tok) lo = mid + 1; else hi = mid;
-      }
-      const size_t src = static_cast<size_t>(o0 + tok) * p.hkv * p.d + c;
-      sk = reinterpret_cast<const uint4*>(p.k_out + src);
-      sv = reinterpret_cast<const uint4*>(p.v_out + src);
-      const bool selected = lo < n_sel && p.sel[s0 + lo] == tok;
-      const size_t dst = selected ? static_cast<size_t>(e0 + n_in + lo) * p.hkv * p.d + c
-                                  : static_cast<size_t>(r0 + tok - lo) * p.hkv * p.d + c;
-      dk = reinterpret_cast<uint4*>((selected ? p.k_ext : p.k_res) + dst);
-      dv = reinterpret_cast<uint4*>((selected ? p.v_ext : p.v_res) + dst);
-    } else {
-      const int t = tok - n_out;
-      const size_t src = static_cast<size_t>(i0 + t) * p.hkv * p.d + c;
-      const size_t dst = static_cast<size_t>(e0 + t) * p.hkv * p.d + c;
-      sk = reinterpret_cast<const uint4*>(p.k_in + src);
-      sv = reinterpret_cast<const uint4*>(p.v_in + src);
-      dk = reinterpret_cast<uint4*>(p.k_ext + dst);
-      dv = reinterpret_cast<uint4*>(p.v_ext + dst);
-    }
-    *dk = *sk;
-    *dv = *sv;
+    const bool blk = row < n_in;
+    const size_t src = blk ? static_cast<size_t>(i0 + row) * p.hkv * p.d + c
+                           : static_cast<size_t>(o0 + p.sel[s0 + row - n_in]) * p.hkv * p.d + c;
+    const size_t dst = static_cast<size_t>(e0 + row) * p.hkv * p.d + c;
+    *reinterpret_cast<uint4*>(p.k_ext + dst) = *reinterpret_cast<const uint4*>((blk ? p.k_in : p.k_out) + src);
+    *reinterpret_cast<uint4*>(p.v_ext + dst) = *reinterpret_cast<const uint4*>((blk ? p.v_in : p.v_out) + src);
   }
 }
 

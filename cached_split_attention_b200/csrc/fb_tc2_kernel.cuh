@@ -336,10 +336,22 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
         if (row_ok) p.cache_l[ce] = l > 0.f ? (m + log2f(l)) * kLn2 : kNegInf;
       };
       if (rec && nB == 0) snapshot();  // empty prefix: (0, -inf)
+      // skip-mask bits of a prefix chunk's 128 keys, loaded one chunk ahead
+      auto skip_of = [&](int c, uint64_t (&w)[2]) {
+        w[0] = w[1] = 0ull;
+        if (p.out_skip && c < nB) {
+          w[0] = skip_bits64(p.out_skip, p.total_out, out0 + c * kN);
+          w[1] = skip_bits64(p.out_skip, p.total_out, out0 + c * kN + 64);
+        }
+      };
+      uint64_t skip_next[2];
+      skip_of(0, skip_next);
       for (int c = 0; c < n_chunks; ++c) {
         const bool seg_out = c < nB;
         const int key0 = seg_out ? c * kN : (c - nB) * kN;
         const int valid = min(kN, (seg_out ? n_out : n_in) - key0);
+        const uint64_t skip[2] = {skip_next[0], skip_next[1]};  // bit k: key key0 + k (+ 64) left out
+        skip_of(c + 1, skip_next);
         // my turn: A(c) follows B(c-1), B(c) follows A(c)
         if ((x == 1 || c > 0) && !__all_sync(0xffffffffu, mbar_wait(&turn[x], (x == 1 ? c : c - 1) & 1))) {
           ok = false;
@@ -366,13 +378,14 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
           reg_fence32(sk[1]);
           reg_fence32(sv[0]);
           reg_fence32(sv[1]);
-          if (valid < kN) {  // ragged last chunk of a segment
+          if (valid < kN || (skip[0] | skip[1])) {  // ragged last chunk of a segment, skipped keys
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
 #pragma unroll
               for (int k = 0; k < 32; ++k) {
-                if (32 * i + k >= valid) sk[i][k] = __float_as_uint(kNegInf);
-                if (64 + 32 * i + k >= valid) sv[i][k] = __float_as_uint(kNegInf);
+                if (32 * i + k >= valid || ((skip[0] >> (32 * i + k)) & 1ull)) sk[i][k] = __float_as_uint(kNegInf);
+                if (64 + 32 * i + k >= valid || ((skip[1] >> (32 * i + k)) & 1ull))
+                  sv[i][k] = __float_as_uint(kNegInf);
               }
             }
           }
@@ -430,7 +443,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
               p1 = ex2(x1);
             }
             rsa[(k >> 1) & 1] = fadd2(rsa[(k >> 1) & 1], f2_pack(p0, p1));
-            pk[k >> 1] = pack_bf16x2(p0, p1);
+            pk[k >> 1] = pack_bf16x2_pos(p0, p1);
           }
           tmem_st16(sp + col, pk);
         };
@@ -442,12 +455,12 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
         tmem_wait_ld();
         reg_fence32(sh[0]);
         reg_fence32(sh[1]);
-        if (valid < kN) {
+        if (valid < kN || skip[1]) {
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
 #pragma unroll
             for (int k = 0; k < 32; ++k)
-              if (64 + 32 * i + k >= valid) sh[i][k] = __float_as_uint(kNegInf);
+              if (64 + 32 * i + k >= valid || ((skip[1] >> (32 * i + k)) & 1ull)) sh[i][k] = __float_as_uint(kNegInf);
           }
         }
         exp_group(sh[0], 32);

@@ -394,7 +394,20 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
         const int r = tid;
         float m = kNegInf, l = 0.f;
         bool ok = true;
+        // skip-mask bits of a prefix chunk's 128 keys, loaded one chunk ahead
+        auto skip_of = [&](int c, uint64_t (&w)[2]) {
+          w[0] = w[1] = 0ull;
+          if (p.out_skip && c >= nA && c < n_local) {
+            const int t0 = out0 + (pa + c - nA) * kN;
+            w[0] = skip_bits64(p.out_skip, p.total_out, t0);
+            w[1] = skip_bits64(p.out_skip, p.total_out, t0 + 64);
+          }
+        };
+        uint64_t skip_next[2];
+        skip_of(0, skip_next);
         for (int c = 0; c < n_local; ++c) {
+          const uint64_t skip[2] = {skip_next[0], skip_next[1]};
+          skip_of(c + 1, skip_next);
           if (c == nA && c > 0) {  // block segment done; the prefix segment starts
             m_in = m;
             l_in = l;
@@ -418,13 +431,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
 #pragma unroll
           for (int i = 0; i < 4; ++i) reg_fence32(sv[i]);
           // Row max of the raw scores (the scale is positive, so it commutes with
-          // the max), four independent chains of 3-input maxima.
-          if (valid < kN) {
+          // the max), four independent chains of 3-input maxima.  Keys past the
+          // segment's end, and prefix keys the skip mask leaves out, get -inf.
+          if (valid < kN || (skip[0] | skip[1])) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
 #pragma unroll
               for (int k = 0; k < 32; ++k)
-                if (32 * i + k >= valid) sv[i][k] = __float_as_uint(kNegInf);
+                if (32 * i + k >= valid || ((skip[i >> 1] >> (32 * (i & 1) + k)) & 1ull))
+                  sv[i][k] = __float_as_uint(kNegInf);
             }
           }
           float mxa[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
@@ -446,7 +461,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
             resc = true;
           }
           const float nm = m == kNegInf ? 0.f : -m;
-          // P = 2^(s * scale - m), rounded to bf16 for the P V product; paired fp32
+          // P = 2^(s * scale - m), rounded to nearest bf16 for the P V product (by
+          // integer arithmetic, pack_bf16x2_pos); paired fp32
           // arithmetic, pairs 8a+0..2 of every eight by the cubic, the rest by MUFU;
           // the row sum in eight chains (four paired accumulators).
           uint32_t pk[2][32];  // packed bf16 pairs: keys 2j, 2j+1 in column j
@@ -470,7 +486,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
                 p1 = ex2(x1);
               }
               rsa[(k >> 1) & 3] = fadd2(rsa[(k >> 1) & 3], f2_pack(p0, p1));
-              pk[i >> 1][(16 * i + k / 2) & 31] = pack_bf16x2(p0, p1);
+              pk[i >> 1][(16 * i + k / 2) & 31] = pack_bf16x2_pos(p0, p1);
             }
           }
           float r0, r1, r2, r3, r4, r5, r6, r7;

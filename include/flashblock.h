@@ -84,6 +84,10 @@ typedef enum fb_status {
  *   cu_seqlens_kv_out [num_seqs+1] offsets of each sequence's prefix (J_out) tokens
  *   cu_seqlens_kv_in  [num_seqs+1] offsets of each sequence's block (J_in) tokens
  * out_splits: number of key splits of the prefix pass; 0 lets the library choose.
+ * kv_out_skip: NULL, or a bitmask over the prefix tokens (device, uint32 words, at least
+ *   ceil(total_kv_out / 32) of them): bit t (bit t % 32 of word t / 32) set leaves prefix
+ *   token t -- row t of k_out / v_out -- out of J_out.  The sparse-residual layout
+ *   (fb_sparse_layout) sets the bits of the keys it moves into the block's key set.
  */
 typedef struct fb_problem {
   int32_t num_seqs, num_heads_q, num_heads_kv, head_dim;
@@ -95,6 +99,7 @@ typedef struct fb_problem {
   int32_t total_q, total_kv_out, total_kv_in; /* host: Q / prefix / block token counts   */
   int32_t max_q, max_kv_out, max_kv_in;       /* host: largest per-sequence count of each */
   int32_t out_splits;
+  const uint32_t* kv_out_skip;
 } fb_problem;
 
 /*
@@ -282,22 +287,26 @@ fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* ca
  *   J_out'(b) = prefix keys of b that are not selected (order kept)
  * cu_sel [num_seqs+1] (device) offsets into sel_idx; sel_idx [total_sel] (device) holds,
  * per sequence, strictly increasing positions in [0, N_b) of the selected prefix keys;
- * total_sel (host) = cu_sel[num_seqs].  Outputs (device, THD bf16, caller-owned):
- *   k_res, v_res [total_kv_out - total_sel, H_kv, d];  k_ext, v_ext [total_kv_in + total_sel, H_kv, d]
- *   cu_seqlens_kv_out_res = cu_seqlens_kv_out - cu_sel, cu_seqlens_kv_in_ext =
- *   cu_seqlens_kv_in + cu_sel ([num_seqs+1] each; may be NULL).
- * The block keeps positions 0..B_b-1 of J_in', so cu_seqlens_q and q_rows stay valid:
- * fb_step on (J_out', J_in') with a cache of total_kv_in + total_sel rows caches the
- * residual and recomputes the selected keys every step; with a fresh cache the result is
- * full attention over prefix and block.  The selection is fixed for a block (a new one
- * changes the residual: refill the cache).  A selection that is not increasing or out of
- * range records FB_ERR_INVALID_ARG on the device (fb_device_status); that sequence is
- * skipped.  At most 65535 sequences per call (FB_ERR_UNSUPPORTED beyond).
+ * total_sel (host) = cu_sel[num_seqs].  Outputs (device, caller-owned):
+ *   k_ext, v_ext [total_kv_in + total_sel, H_kv, d] (THD bf16): J_in' of every sequence;
+ *   kv_out_skip [ceil(total_kv_out / 32)] uint32: the bitmask of the selected prefix
+ *     tokens (bit t of the global prefix row t), cleared and set by this call;
+ *   cu_seqlens_kv_in_ext = cu_seqlens_kv_in + cu_sel ([num_seqs+1]; may be NULL).
+ * The residual prefix is not copied: J_out' is the prefix (k_out, v_out,
+ * cu_seqlens_kv_out unchanged) with kv_out_skip set in the problem, which every prefix
+ * pass honours.  The block keeps positions 0..B_b-1 of J_in', so cu_seqlens_q and q_rows
+ * stay valid: fb_step on that problem (cu_seqlens_kv_in_ext, kv_out_skip) with a cache of
+ * total_kv_in + total_sel rows caches the residual and recomputes the selected keys every
+ * step; with a fresh cache the result is full attention over prefix and block.  The
+ * selection is fixed for a block (a new one changes the residual: refill the cache).
+ * The pass moves the block rows and the selected rows only.  A selection that is not
+ * increasing or out of range records FB_ERR_INVALID_ARG on the device (fb_device_status);
+ * that sequence is skipped.  At most 65535 sequences per call (FB_ERR_UNSUPPORTED beyond).
  */
 fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, const int32_t* sel_idx,
                            int32_t total_sel, const fb_bf16* k_out, const fb_bf16* v_out, const fb_bf16* k_in,
-                           const fb_bf16* v_in, fb_bf16* k_res, fb_bf16* v_res, fb_bf16* k_ext, fb_bf16* v_ext,
-                           int32_t* cu_seqlens_kv_out_res, int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream);
+                           const fb_bf16* v_in, fb_bf16* k_ext, fb_bf16* v_ext, uint32_t* kv_out_skip,
+                           int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream);
 
 /*
  * Block transition (FlashBlock, gist.science/es/paper/2602.05305, "Mecanismo Central": a

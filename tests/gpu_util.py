@@ -52,7 +52,7 @@ def workspace_for(steps_problems, out_splits=0, device="cuda"):
 
 
 def run_policy_gpu(w, flags=None, out_splits=0, head_reuse_in=None, device="cuda", keep=True, cache=None,
-                   k_out=None, v_out=None):
+                   k_out=None, v_out=None, kv_out_skip=None):
     """Run a workload's steps through fb_step (on ``cache`` when given, else on a new
     empty one; on the device prefix ``k_out``/``v_out`` when given, else on w's
     uploaded); returns per-step dicts of numpy arrays and the cache."""
@@ -67,7 +67,7 @@ def run_policy_gpu(w, flags=None, out_splits=0, head_reuse_in=None, device="cuda
     out = []
     for s, st in enumerate(w.steps):
         p = st.problem
-        dp = B.DeviceProblem(p, device, out_splits)
+        dp = B.DeviceProblem(p, device, out_splits, kv_out_skip=kv_out_skip)
         q = B.bf16_tensor(st.q, device)
         k_in = B.bf16_tensor(st.k_in, device)
         v_in = B.bf16_tensor(st.v_in, device)

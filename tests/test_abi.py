@@ -38,7 +38,8 @@ def test_library_exports_every_declared_symbol():
 def _problem(B, **kw):
     args = dict(num_seqs=1, num_heads_q=32, num_heads_kv=32, head_dim=128, softmax_scale=0.088,
                 cu_seqlens_q=16, q_rows=0, cu_seqlens_kv_out=16, cu_seqlens_kv_in=16, total_q=32,
-                total_kv_out=4096, total_kv_in=32, max_q=32, max_kv_out=4096, max_kv_in=32, out_splits=0)
+                total_kv_out=4096, total_kv_in=32, max_q=32, max_kv_out=4096, max_kv_in=32, out_splits=0,
+                kv_out_skip=None)
     args.update(kw)
     return B.FbProblem(**args)
 
@@ -98,13 +99,20 @@ def test_host_validation_without_gpu():
     assert B._lib.fb_cache_copy_seq(ctypes.byref(ok), ctypes.byref(cache5), 0, 3, None) == B.ERR_INVALID_ARG
     assert "out of range" in B.last_error()
     assert B._lib.fb_cache_copy_seq(ctypes.byref(ok), ctypes.byref(cache5), 0, 0, None) == B.OK  # no-op
-    rc = B._lib.fb_sparse_layout(ctypes.byref(ok), 16, 16, 5000, 16, 16, 16, 16, 16, 16, 16, 16, None, None, None)
+    rc = B._lib.fb_sparse_layout(ctypes.byref(ok), 16, 16, 5000, 16, 16, 16, 16, 16, 16, 16, None, None)
     assert rc == B.ERR_INVALID_ARG and "total_sel" in B.last_error()
-    rc = B._lib.fb_sparse_layout(ctypes.byref(ok), None, 16, 4, 16, 16, 16, 16, 16, 16, 16, 16, None, None, None)
+    rc = B._lib.fb_sparse_layout(ctypes.byref(ok), None, 16, 4, 16, 16, 16, 16, 16, 16, 16, None, None)
     assert rc == B.ERR_INVALID_ARG and "cu_sel" in B.last_error()
     many = _problem(B, num_seqs=70000, total_q=0, max_q=0, total_kv_in=0, max_kv_in=0, total_kv_out=0, max_kv_out=0)
-    rc = B._lib.fb_sparse_layout(ctypes.byref(many), 16, 16, 0, 16, 16, 16, 16, 16, 16, 16, 16, None, None, None)
+    rc = B._lib.fb_sparse_layout(ctypes.byref(many), 16, 16, 0, 16, 16, 16, 16, 16, 16, 16, None, None)
     assert rc == B.ERR_UNSUPPORTED and "65535" in B.last_error()
+    rc = B._lib.fb_sparse_layout(ctypes.byref(ok), 16, 16, 4, 16, 16, 16, 16, 16, 16, None, None, None)
+    assert rc == B.ERR_INVALID_ARG and "kv_out_skip" in B.last_error()
+    rc = B._lib.fb_sparse_layout(ctypes.byref(ok), 16, 16, 4, 16, 16, 16, 16, 16, 16, 18, None, None)
+    assert rc == B.ERR_INVALID_ARG and "aligned" in B.last_error()
+    skewed = _problem(B, kv_out_skip=18)
+    assert B._lib.fb_workspace_size(ctypes.byref(skewed), ctypes.byref(n)) == B.ERR_INVALID_ARG
+    assert "kv_out_skip" in B.last_error()
     # block transition: in place only for one sequence, K and V alike
     two = _problem(B, num_seqs=2)
     rc = B._lib.fb_prefix_append(ctypes.byref(two), 16, 32, 48, 64, 16, 32, None, None)

@@ -68,8 +68,9 @@ def test_extension_row_byte_models():
     assert bench.cache_copy_bytes(p, 5, 4, with_q_ref=True) == 2 * 64 * 32 * 772 + 2 * 32 * 5
     assert bench.cache_copy_bytes(p, 0, 5, with_q_ref=False) == 2 * 4 * 32 * 516 + 2 * 32 * 5
     q = W.long_context_gqa(steps=1, batch=2, prefix=1000, heads_q=8, heads_kv=2).problem
-    # (2000 prefix + 128 block rows) x 2 heads x 128 x bf16 x (K, V), read and written, + indices
-    assert bench.sparse_layout_bytes(q, 10) == 2 * 2128 * 2 * 128 * 2 * 2 + 4 * (10 + 9)
+    # (128 block + 10 selected rows) x 2 heads x 128 x bf16 x (K, V), read and written,
+    # + the skip mask (2000 prefix tokens: 63 words) + indices
+    assert bench.sparse_layout_bytes(q, 10) == 2 * 138 * 2 * 128 * 2 * 2 + 4 * 63 + 4 * (10 + 9)
 
 
 def test_sparse_selection_shape():
