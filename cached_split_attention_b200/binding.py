@@ -142,7 +142,12 @@ class DeviceProblem:
         self.kv_out_skip = kv_out_skip
         mk = lambda a: torch.as_tensor(np.ascontiguousarray(a, dtype=np.int32)).to(device)
         self.cu_q = mk(problem.cu_seqlens_q)
-        self.q_rows = mk(problem.q_rows) if len(problem.q_rows) else None
+        # NULL q_rows means "row r of sequence b is block position r - cu_seqlens_q[b]"
+        # (flashblock.h): passed when the active rows are exactly that
+        starts = np.repeat(np.asarray(problem.cu_seqlens_q[:-1], dtype=np.int64), np.diff(problem.cu_seqlens_q))
+        identity = np.array_equal(np.asarray(problem.q_rows, dtype=np.int64),
+                                  np.arange(len(problem.q_rows), dtype=np.int64) - starts)
+        self.q_rows = mk(problem.q_rows) if len(problem.q_rows) and not identity else None
         self.cu_out = mk(problem.cu_seqlens_kv_out)
         self.cu_in = mk(problem.cu_seqlens_kv_in)
         self.struct = FbProblem(

@@ -189,21 +189,12 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = fals
     if (p->out_splits > 0) {
       splits = p->out_splits;
     } else {
-      // The split with the shortest makespan: S CTAs per group take ceil(G S /
-      // slots) waves of 1/S of a group's keys each, and every further split adds
-      // about 3 % for its partial's merge.  One wave when G <= slots: S = slots / G.
+      // One wave: as many CTAs per group as the resident slots allow.  (A split
+      // chosen by makespan -- more waves of shorter CTAs -- was measured slower:
+      // the per-CTA lead-in and merge outweigh the better packing of the waves.)
       const int per_sm = std::max(1, std::min(233472 / (pl.smem + 1024), 2048 / pl.threads));
       const long slots = static_cast<long>(num_sms) * per_sm;
-      const long G = std::max(1, pl.n_groups);
-      double best = 1e30;
-      for (int s = 1; s <= fb::kMaxSplits; ++s) {
-        const double waves = static_cast<double>((G * s + slots - 1) / slots);
-        const double span = waves / s * (1.0 + 0.03 * (s - 1));
-        if (span < best - 1e-9) {
-          best = span;
-          splits = s;
-        }
-      }
+      splits = static_cast<int>(std::max(1L, slots / std::max(1, pl.n_groups)));
     }
     splits = std::max(1, std::min({splits, fb::kMaxSplits, chunks}));
   }

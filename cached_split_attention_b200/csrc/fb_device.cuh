@@ -209,14 +209,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Two non-negative finite floats -> packed bf16x2, rounded to nearest (ties away
-// from zero) with integer arithmetic: half a bf16 ulp (0x8000) is added to the
-// fp32 bits and the high halves are kept.  Two adds and a byte permute on the ALU
-// instead of a conversion on the XU pipe, which the softmax's exponentials share.
-__device__ __forceinline__ uint32_t pack_bf16x2_pos(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
 __device__ __forceinline__ float quad_max(float v) {
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));

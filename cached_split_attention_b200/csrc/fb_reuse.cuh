@@ -107,7 +107,8 @@ __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b
       const size_t ce = static_cast<size_t>(in0 + pos) * p.hq + (fe % p.hq);
       mbar_arrive_expect_tx(bar, D * 4);
       bulk_load_1d(ca_s + tid * kCS, p.cache_a + ce * D, D * 4, bar);
-      cl_s[tid] = p.cache_l[ce];
+      cp_async_4(cl_s + tid, p.cache_l + ce);
+      cp_async_commit();
     }
   } else if (tid < nr16) {
 #pragma unroll
@@ -121,6 +122,7 @@ __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b
     if (tid == 0) record_status(kDevTimeout);
     mbar_wait(bar, 0);
   }
+  cp_async_wait_all();  // the row's L_out
   __syncthreads();
   if (!ok) return;
 

@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
               p1 = ex2(x1);
             }
             rsa[(k >> 1) & 1] = fadd2(rsa[(k >> 1) & 1], f2_pack(p0, p1));
-            pk[k >> 1] = pack_bf16x2_pos(p0, p1);
+            pk[k >> 1] = pack_bf16x2(p0, p1);
           }
           tmem_st16(sp + col, pk);
         };

@@ -461,8 +461,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
             resc = true;
           }
           const float nm = m == kNegInf ? 0.f : -m;
-          // P = 2^(s * scale - m), rounded to nearest bf16 for the P V product (by
-          // integer arithmetic, pack_bf16x2_pos); paired fp32
+          // P = 2^(s * scale - m), rounded to bf16 for the P V product; paired fp32
           // arithmetic, pairs 8a+0..2 of every eight by the cubic, the rest by MUFU;
           // the row sum in eight chains (four paired accumulators).
           uint32_t pk[2][32];  // packed bf16 pairs: keys 2j, 2j+1 in column j
@@ -486,7 +485,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
                 p1 = ex2(x1);
               }
               rsa[(k >> 1) & 3] = fadd2(rsa[(k >> 1) & 3], f2_pack(p0, p1));
-              pk[i >> 1][(16 * i + k / 2) & 31] = pack_bf16x2_pos(p0, p1);
+              pk[i >> 1][(16 * i + k / 2) & 31] = pack_bf16x2(p0, p1);
             }
           }
           float r0, r1, r2, r3, r4, r5, r6, r7;
