@@ -369,7 +369,7 @@ def _elapsed_us(ev):
 # built from.
 KERNEL_OF = {"dllm_layer": "attn_kernel", "tiny": "attn_kernel", "long_context_gqa": "tc_attn_kernel",
              "varlen_branches": "tc_attn_kernel", "video": "tc2_attn_kernel"}
-_BASE_SOURCES = ("fb_device.cuh", "fb_kernels.cuh")
+_BASE_SOURCES = ("fb_device.cuh", "fb_kernels.cuh", "fb_reuse.cuh")
 KERNEL_SOURCES = {"attn_kernel": _BASE_SOURCES,
                   "tc_attn_kernel": _BASE_SOURCES + ("fb_tcgen05.cuh", "fb_tc_kernel.cuh"),
                   "tc2_attn_kernel": _BASE_SOURCES + ("fb_tcgen05.cuh", "fb_tc_kernel.cuh", "fb_tc2_kernel.cuh")}

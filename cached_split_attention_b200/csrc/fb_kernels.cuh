@@ -105,6 +105,25 @@ struct alignas(64) Params {
   int lean;          // 1: groups whose heads all reuse take the lean path
 };
 
+// Bring the kernel's tensor-map descriptors on chip while the previous kernel of
+// the stream finishes (they live in this launch's parameters, which no earlier
+// kernel writes, so this may run before pdl_wait).
+__device__ __forceinline__ void prefetch_maps(const Params& p) {
+  if (threadIdx.x != 0) return;
+  if (p.total_out > 0) {
+    prefetch_tensormap(&p.tm_k_out);
+    prefetch_tensormap(&p.tm_v_out);
+  }
+  if (p.total_in > 0) {
+    prefetch_tensormap(&p.tm_k_in);
+    prefetch_tensormap(&p.tm_v_in);
+    if (p.lean) {
+      prefetch_tensormap(&p.tm_k_lean);
+      prefetch_tensormap(&p.tm_v_lean);
+    }
+  }
+}
+
 // Reuse decision of (b, h); see fb_step in flashblock.h.
 __device__ __forceinline__ bool head_recompute(const Params& p, int b, int h) {
   const int idx = b * p.hq + h;
@@ -406,6 +425,7 @@ namespace fb {
 
 template <int D, int WM, int WN, int STAGES>
 __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kernel(const __grid_constant__ Params p) {
+  prefetch_maps(p);
   pdl_wait();
   pdl_trigger();
   using C = Cfg<D, WM, WN, STAGES>;
@@ -764,6 +784,14 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
         const int j = rho % g;
         float kind = 0.f;
         float lo2 = kNegInf, li2 = kNegInf;
+        // the block partial's normalisers first: their loads go out with the prefix's
+        float l2i[kInE];
+#pragma unroll
+        for (int w = 0; w < kInE; ++w) {
+          l2i[w] = kNegInf;
+          if (p.do_in && pos >= 0 && w < n_in_e)
+            l2i[w] = (cluster_mode ? ld_f(in_a, S - 1, C::kPartL + r) : in_part[C::kPartL + w * TR + r]) * kLog2e;
+        }
         if (pos >= 0) {
           const int ce = (in0 + pos) * p.hq + hk * g + j;
           wr[kOutE + kInE + 4] = __int_as_float(ce);
@@ -784,16 +812,7 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
           } else {
             kind = 3.f;  // block pass alone
           }
-          if (p.do_in) {
-            float l2[kInE];
-#pragma unroll
-            for (int w = 0; w < kInE; ++w) {
-              l2[w] = kNegInf;
-              if (w < n_in_e)
-                l2[w] = (cluster_mode ? ld_f(in_a, S - 1, C::kPartL + r) : in_part[C::kPartL + w * TR + r]) * kLog2e;
-            }
-            li2 = log2_weights<kInE>(l2, wr + kOutE);
-          }
+          if (p.do_in) li2 = log2_weights<kInE>(l2i, wr + kOutE);
         }
         float wo = 1.f, lf2 = li2;
         if (p.fused && pos >= 0) {
@@ -827,6 +846,17 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
         if (kind == 0) continue;
         const size_t ce = static_cast<unsigned>(__float_as_int(wr[kOutE + kInE + 4]));
         const size_t fe = static_cast<unsigned>(__float_as_int(wr[kOutE + kInE + 5]));
+        // every load of the item is issued before its stores (a load after a
+        // store to a generic address would wait for it)
+        float4 vi[kInE];
+        if (p.do_in) {
+#pragma unroll
+          for (int w = 0; w < kInE; ++w) {
+            if (w >= n_in_e) continue;
+            vi[w] = cluster_mode ? ld_f4(in_a, S - 1, r * C::kPStride + c4)
+                                 : *reinterpret_cast<const float4*>(in_part + (w * TR + r) * C::kPStride + c4);
+          }
+        }
         float4 ao = make_float4(0.f, 0.f, 0.f, 0.f);
         if (kind == 1) {
           float4 v[kOutE];
@@ -839,26 +869,21 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
 #pragma unroll
           for (int k = 0; k < kOutE; ++k)
             if (wr[k] != 0.f) fma4(ao, wr[k], v[k]);
-          *reinterpret_cast<float4*>(p.cache_a + ce * D + c4) = ao;
-          if (c4 == 0) p.cache_l[ce] = wr[kOutE + kInE + 1];
         } else if (kind == 2) {
           ao = C::kStageCache ? *reinterpret_cast<const float4*>(cache_s + r * C::kPStride + c4)
                               : *reinterpret_cast<const float4*>(p.cache_a + ce * D + c4);
         }
-        if (!p.do_in) continue;
         float4 ai = make_float4(0.f, 0.f, 0.f, 0.f);
-        {
-          float4 v[kInE];
-#pragma unroll
-          for (int w = 0; w < kInE; ++w) {
-            if (w >= n_in_e) continue;
-            v[w] = cluster_mode ? ld_f4(in_a, S - 1, r * C::kPStride + c4)
-                                : *reinterpret_cast<const float4*>(in_part + (w * TR + r) * C::kPStride + c4);
-          }
+        if (p.do_in) {
 #pragma unroll
           for (int w = 0; w < kInE; ++w)
-            if (w < n_in_e) fma4(ai, wr[kOutE + w], v[w]);
+            if (w < n_in_e) fma4(ai, wr[kOutE + w], vi[w]);
         }
+        if (kind == 1) {
+          *reinterpret_cast<float4*>(p.cache_a + ce * D + c4) = ao;
+          if (c4 == 0) p.cache_l[ce] = wr[kOutE + kInE + 1];
+        }
+        if (!p.do_in) continue;
         if (!p.fused) {
           *reinterpret_cast<float4*>(p.a_in + fe * D + c4) = ai;
           if (c4 == 0) p.l_in[fe] = wr[kOutE + kInE + 2];

@@ -139,36 +139,46 @@ __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b
       const uint32_t vb = smem_u32(vs + (k0 / kBN) * kT);
       consume_keys<D, 32>(acc, qf, kb, vb, k0 % kBN, k0, n_in, p.scale_log2, lane);
     }
+    // Merge weights of the thread's two rows first (independent chains), then
+    // each row's columns: all of its cached values are loaded before any store
+    // (the loads would otherwise wait behind the stores of earlier columns).
+    float wo[2], wz[2], lf[2];
+    int er[2];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const float z = quad_sum(acc.l[i]);
       const int r = 16 * slab + (lane >> 2) + 8 * i;
-      const int e = fe_s[r];
-      if (e < 0) continue;
+      er[i] = fe_s[r];
       const float li2 = z > 0.f ? acc.m[i] + lg2_approx(z) : kNegInf;
       const float lo_nat = cl_s[r];
       const float lo2 = lo_nat == kNegInf ? kNegInf : lo_nat * kLog2e;
       const float m2 = fmaxf(lo2, li2);
-      float wo = 0.f, wi = 0.f, lf2 = kNegInf;
+      float w_o = 0.f, w_i = 0.f, lf2 = kNegInf;
       if (m2 != kNegInf) {
-        wo = lo2 == kNegInf ? 0.f : ex2(lo2 - m2);
-        wi = li2 == kNegInf ? 0.f : ex2(li2 - m2);
-        const float inv = rcp_approx(wo + wi);
-        lf2 = m2 + lg2_approx(wo + wi);
-        wo *= inv;
-        wi *= inv;
+        w_o = lo2 == kNegInf ? 0.f : ex2(lo2 - m2);
+        w_i = li2 == kNegInf ? 0.f : ex2(li2 - m2);
+        const float inv = rcp_approx(w_o + w_i);
+        lf2 = m2 + lg2_approx(w_o + w_i);
+        w_o *= inv;
+        w_i *= inv;
       }
-      const float wz = z > 0.f ? wi * rcp_approx(z) : 0.f;  // A_in = O / z
-      const float* crow = ca_s + r * kCS;
-      __nv_bfloat16* dst = p.a_full + static_cast<size_t>(e) * D;
+      wo[i] = w_o;
+      wz[i] = z > 0.f ? w_i * rcp_approx(z) : 0.f;  // A_in = O / z
+      lf[i] = lf2 == kNegInf ? kNegInf : lf2 * kLn2;
+    }
 #pragma unroll
-      for (int n = 0; n < D / 8; ++n) {
-        const int col = n * 8 + 2 * (lane & 3);
-        const float2 ao = *reinterpret_cast<const float2*>(crow + col);
-        *reinterpret_cast<__nv_bfloat162*>(dst + col) = __floats2bfloat162_rn(
-            fmaf(wo, ao.x, wz * acc.o[n][2 * i]), fmaf(wo, ao.y, wz * acc.o[n][2 * i + 1]));
-      }
-      if ((lane & 3) == 0 && p.l_full) p.l_full[e] = lf2 == kNegInf ? kNegInf : lf2 * kLn2;
+    for (int i = 0; i < 2; ++i) {
+      if (er[i] < 0) continue;
+      const float* crow = ca_s + (16 * slab + (lane >> 2) + 8 * i) * kCS + 2 * (lane & 3);
+      float2 ao[D / 8];
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) ao[n] = *reinterpret_cast<const float2*>(crow + n * 8);
+      __nv_bfloat16* dst = p.a_full + static_cast<size_t>(er[i]) * D + 2 * (lane & 3);
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n)
+        *reinterpret_cast<__nv_bfloat162*>(dst + n * 8) = __floats2bfloat162_rn(
+            fmaf(wo[i], ao[n].x, wz[i] * acc.o[n][2 * i]), fmaf(wo[i], ao[n].y, wz[i] * acc.o[n][2 * i + 1]));
+      if ((lane & 3) == 0 && p.l_full) p.l_full[er[i]] = lf[i];
     }
   }
 }

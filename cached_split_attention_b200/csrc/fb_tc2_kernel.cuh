@@ -61,6 +61,7 @@ static_assert(kSmem <= 232448, "shared memory per CTA");
 }  // namespace tc2
 
 __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid_constant__ Params p) {
+  prefetch_maps(p);
   pdl_wait();
   pdl_trigger();
   using namespace tc2;

@@ -118,6 +118,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }  // namespace tc
 
 __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_constant__ Params p) {
+  prefetch_maps(p);
   pdl_wait();
   pdl_trigger();
   using namespace tc;
@@ -687,6 +688,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
           if (kind == 2) {
             const size_t ce = static_cast<unsigned>(__float_as_int(wr[kW0 + 4]));
             ao[u] = *reinterpret_cast<const float4*>(p.cache_a + ce * kD + c4);
+          } else if (kind == 1) {  // the prefix partials of the row, combined here (before any store)
+#pragma unroll
+            for (int k = 0; k < kMaxSplits; ++k)
+              if (wr[k] != 0.f) fma4(ao[u], wr[k], ld_f4(out_a, k, r * kPStride + c4));
           }
           if (kind != 0 && p.do_in && wr[kMaxSplits] != 0.f) ai[u] = ld_f4(in_a, in_rank, r * kPStride + c4);
         }
@@ -702,13 +707,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
           const size_t ce = static_cast<unsigned>(__float_as_int(wr[kW0 + 4]));
           const size_t fe = static_cast<unsigned>(__float_as_int(wr[kW0 + 5]));
           if (kind == 1) {
-            float4 v[kMaxSplits];
-#pragma unroll
-            for (int k = 0; k < kMaxSplits; ++k)
-              if (wr[k] != 0.f) v[k] = ld_f4(out_a, k, r * kPStride + c4);
-#pragma unroll
-            for (int k = 0; k < kMaxSplits; ++k)
-              if (wr[k] != 0.f) fma4(ao[u], wr[k], v[k]);
             *reinterpret_cast<float4*>(p.cache_a + ce * kD + c4) = ao[u];
             if (c4 == 0) p.cache_l[ce] = wr[kW0 + 1];
           }
