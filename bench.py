@@ -469,7 +469,7 @@ def measure(name, args, world, rank, local, device):
     hbm_peak = float(peaks.get("hbm_gbs", 6650.0))
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
     kernel = KERNEL_OF[name]
-    traffic = None
+    traffic = traffic_alg = None
     try:
         prof = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
         for ent in prof.get("entries", []):
@@ -477,6 +477,7 @@ def measure(name, args, world, rank, local, device):
             if (ent.get("workload") == name and ent.get("kernel") == kernel
                     and ent.get("kernel_source_sha256") == kernel_source_digest(kernel)):
                 traffic = ent.get("dram_bytes_per_recompute_launch")
+                traffic_alg = ent.get("algorithmic_bytes_of_that_launch")
     except Exception:
         pass
     # the video block is a dense contraction (about 1500 flop per byte): its bound
@@ -543,6 +544,9 @@ def measure(name, args, world, rank, local, device):
              {"bound": "hbm", "achieved": round(ach_rec, 1), "peak": hbm_peak, "unit": "GB/s",
               "frac": round(ach_rec / hbm_peak, 4), "peak_source": peak_src}),
             kernel=f"{kernel}, recompute launches (prefix + block pass + merge)", traffic=traffic,
+            # the captured launch recomputes every head; the episode's recompute
+            # launches may recompute fewer (gated heads), so compare with this
+            traffic_launch_algorithmic_bytes=traffic_alg,
             algorithmic_bytes_per_launch=round(float(np.mean(bytes_rec))) if rec_steps else None,
             algorithmic_flops_per_launch=round(float(np.mean(flops_rec))) if rec_steps else None,
             launches=len(rec_steps) * L * args.steps),
