@@ -52,9 +52,19 @@ __host__ __device__ constexpr int smem_bytes(int d, int chunks, int rows) {
 // rho % g) of the sequence's packed active tokens -- with the block keys of b.
 // Every thread of the CTA calls it (it has CTA barriers); `smem` is the kernel's
 // 1024-byte aligned dynamic shared memory.
+// Block position of the lean row thread `tid` owns among rows [r0, r0 + nr) (-1:
+// none).  Read from q_rows before the kernel waits for the previous kernel of the
+// stream (index arrays are not written by any kernel that lets this one start
+// early); the caller has checked the sequence's ranges against the host totals.
+__device__ __forceinline__ int lean_pos(const Params& p, int q0, int r0, int nr, int tid) {
+  if (tid >= nr) return -1;
+  const int tok = (r0 + tid) / p.g;
+  return p.q_rows ? p.q_rows[q0 + tok] : tok;
+}
+
 template <int D>
 __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b, int hk, int q0, int in0, int n_in,
-                                           int r0, int nr, int tid, int nthreads) {
+                                           int r0, int nr, int pos_pre, int tid, int nthreads) {
   constexpr int kT = reuse::tile_bytes(D);
   constexpr int kQS = reuse::q_stride(D);
   constexpr int kCS = reuse::c_stride(D);
@@ -72,13 +82,12 @@ __device__ __forceinline__ void lean_reuse(const Params& p, uint8_t* smem, int b
   const int lane = tid & 31;
   const int used = (n_in + kBN - 1) / kBN;  // 64-key chunks holding the block
 
-  // One thread per row reads its block position (the cache entry depends on it);
+  // One thread per row has its block position (read before the dependency wait);
   // thread 0 arms the barrier: one arrival per row, one for the block K/V.
-  int pos = -1, fe = -1;
+  int pos = pos_pre, fe = -1;
   if (tid < nr) {
     const int rho = r0 + tid;
     const int tok = rho / g;
-    pos = p.q_rows ? p.q_rows[q0 + tok] : tok;
     fe = (q0 + tok) * p.hq + hk * g + (rho - tok * g);
   }
   if (tid == 0) {

@@ -35,7 +35,8 @@ struct SparseParams {
 // x-block also sets the skip bits of the selected tokens.
 __global__ void __launch_bounds__(256) sparse_layout_kernel(const SparseParams p) {
   pdl_wait();
-  pdl_trigger();
+  // no early launch of the next kernel: it may read what this one writes (index
+  // arrays, K/V) before its own dependency wait
   const int b = blockIdx.y;
   const int o0 = p.cu_out[b], n_out = p.cu_out[b + 1] - o0;
   const int i0 = p.cu_in[b], n_in = p.cu_in[b + 1] - i0;

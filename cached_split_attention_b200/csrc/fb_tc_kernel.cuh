@@ -119,8 +119,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_constant__ Params p) {
   prefetch_maps(p);
-  pdl_wait();
-  pdl_trigger();
   using namespace tc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -154,14 +152,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   const int g = p.g;
 
   // ------------------------------------------------------------ group metadata
+  // Index arrays before the wait for the previous kernel of the stream (see
+  // attn_kernel); the cache state after it.
   const int q0 = p.cu_q[b];
   const int n_q = p.cu_q[b + 1] - q0;
   const int out0 = p.cu_out[b];
   const int n_out = p.cu_out[b + 1] - out0;
   const int in0 = p.cu_in[b];
   const int n_in = p.cu_in[b + 1] - in0;
-  if (tid < g) s_rec[tid] = head_recompute(p, b, hk * g + tid) ? 1 : 0;
-  const bool need_state = state_vote(p, tid, kThreads);
   const bool ranges_ok = q0 >= 0 && n_q >= 0 && q0 + n_q <= p.total_q && out0 >= 0 && n_out >= 0 &&
                          out0 + n_out <= p.total_out && in0 >= 0 && n_in >= 0 && in0 + n_in <= p.total_in &&
                          n_q <= n_in;
@@ -169,6 +167,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   if (!ranges_ok && tid == 0 && t == 0 && split == 0) record_status(kDevBadIndex);
   const int rows = ranges_ok ? n_q * g : 0;
   const int nrows = max(0, min(kM, rows - row0));
+  int lean_r0 = 0, lean_nr = 0, lean_p = -1;  // this CTA's rows on the lean path, and its thread's position
+  if (p.lean && nrows > 0) {
+    lean_rows(nrows, split, S, lean_r0, lean_nr);
+    lean_p = lean_pos(p, q0, row0 + lean_r0, lean_nr, tid);
+  }
+  pdl_wait();
+  pdl_trigger();
+  if (tid < g) s_rec[tid] = head_recompute(p, b, hk * g + tid) ? 1 : 0;
+  const bool need_state = state_vote(p, tid, kThreads);
   bool any_rec = false;
   for (int j = 0; j < g; ++j) any_rec |= (s_rec[j] != 0);
 
@@ -191,12 +198,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   // A group whose heads all reuse takes the lean reuse path (its CTAs share the rows).
   const bool lean = p.lean && !any_rec && active;
   if (lean) {
-    int r0, nr;
-    lean_rows(nrows, split, S, r0, nr);
     if (n_in > p.reuse_chunks * kBN) {
       if (tid == 0) record_status(kDevBadIndex);
-    } else if (nr > 0) {
-      lean_reuse<kD>(p, smem, b, hk, q0, in0, n_in, row0 + r0, nr, tid, kThreads);
+    } else if (lean_nr > 0) {
+      lean_reuse<kD>(p, smem, b, hk, q0, in0, n_in, row0 + lean_r0, lean_nr, lean_p, tid, kThreads);
     }
   } else if (active && (has_in || has_out || cluster_mode)) {
     // -------------------------------------------------------- Q rows (before the K/V stream)

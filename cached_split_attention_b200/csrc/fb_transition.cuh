@@ -30,7 +30,8 @@ struct AppendParams {
 // the sequence's prefix rows (when copied) then its block rows.
 __global__ void __launch_bounds__(256) prefix_append_kernel(const AppendParams p) {
   pdl_wait();
-  pdl_trigger();
+  // no early launch of the next kernel: it may read what this one writes (index
+  // arrays, K/V) before its own dependency wait
   const int b = blockIdx.y;
   const int o0 = p.cu_out[b], n_out = p.cu_out[b + 1] - o0;
   const int i0 = p.cu_in[b], n_in = p.cu_in[b + 1] - i0;

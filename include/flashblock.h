@@ -84,6 +84,13 @@ typedef enum fb_status {
  *   cu_seqlens_kv_out [num_seqs+1] offsets of each sequence's prefix (J_out) tokens
  *   cu_seqlens_kv_in  [num_seqs+1] offsets of each sequence's block (J_in) tokens
  * out_splits: number of key splits of the prefix pass; 0 lets the library choose.
+ * Ordering: the attention calls read the index arrays (cu_seqlens_*, q_rows) before they
+ *   wait for the previous kernel of the stream to finish, so that these loads overlap its
+ *   tail.  A kernel that precedes such a call on its stream and lets its dependents launch
+ *   early (programmatic dependent launch, griddepcontrol.launch_dependents) must not write
+ *   them; ordinary kernels and copies are waited for as usual.  The library's own kernels
+ *   that write index arrays (fb_sparse_layout, fb_prefix_append) do not launch dependents
+ *   early.  Everything else (Q/K/V, the cache, kv_out_skip) is read after the wait.
  * kv_out_skip: NULL, or a bitmask over the prefix tokens (device, uint32 words, at least
  *   ceil(total_kv_out / 32) of them): bit t (bit t % 32 of word t / 32) set leaves prefix
  *   token t -- row t of k_out / v_out -- out of J_out.  The sparse-residual layout
