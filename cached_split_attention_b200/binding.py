@@ -57,7 +57,7 @@ class FbParams(ctypes.Structure):
 class FbPlanInfo(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("kernel", "rows_per_tile", "tiles", "work_items", "splits", "ctas",
                                               "threads", "smem_bytes", "keys_per_chunk", "num_sms",
-                                              "lean_reuse", "lean_smem_bytes")]
+                                              "lean_reuse", "lean_smem_bytes", "lean_early")]
 
 
 def _load():

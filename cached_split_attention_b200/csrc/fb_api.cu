@@ -101,7 +101,8 @@ struct Plan {
   int order_items = 0;  // work items of the two-tile kernel (0: the problem never takes it)
   // lean reuse path (fused step, blocks of at most reuse::kMaxKeys keys)
   bool reuse = false;
-  int reuse_chunks = 0, reuse_smem = 0;
+  int reuse_chunks = 0, reuse_smem = 0, reuse_bt = 0;
+  bool reuse_early = false;  // every CTA resident at once: lean loads before the decision
 };
 
 int device_sms() {
@@ -201,13 +202,21 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = fals
   pl.splits = splits;
   // Lean reuse path: blocks of up to 128 keys, when the kernel's shared memory
   // holds the block K/V and a tile of rows with their cache entries.
-  if (fused && !pl.tc2 && p->max_kv_in > 0 && p->max_kv_in <= fb::reuse::kMaxKeys) {
+  if (fused && !pl.tc2 && p->max_kv_in > 0 && p->max_kv_in <= fb::reuse::kMaxKeys && rows > 0) {
     const int chunks = (p->max_kv_in + fb::kBN - 1) / fb::kBN;
-    const int need = fb::reuse::smem_bytes(pl.d, chunks, (pl.tr + 15) / 16 * 16) + 1024;
-    if (need <= pl.smem) {
+    // most rows a CTA takes (lean_rows: whole 16-row slabs shared by the splits)
+    const int slabs = static_cast<int>((std::min<long>(pl.tr, rows) + 15) / 16);
+    const int nr_max = (slabs + pl.splits - 1) / pl.splits * 16;
+    const int bt = fb::reuse::box_tokens(pl.g, nr_max);
+    const int need = fb::reuse::smem_bytes(pl.d, chunks, pl.g, bt) + 1024;
+    // TMA box extents are at most 256; a box token's thread is one of warps 1..
+    if (need <= pl.smem && pl.g <= 256 && bt <= 256 && bt <= pl.threads - fb::kLeanTok0) {
+      const int per_sm = std::max(1, std::min(233472 / (pl.smem + 1024), 2048 / pl.threads));
       pl.reuse = true;
       pl.reuse_chunks = chunks;
       pl.reuse_smem = need;
+      pl.reuse_bt = bt;
+      pl.reuse_early = static_cast<long>(pl.n_groups) * pl.splits <= static_cast<long>(num_sms) * per_sm;
     }
   }
   // workspace layout
@@ -274,6 +283,39 @@ fb_status kv_map(const void* ptr, int tokens, int hkv, int d, int box_rows, CUte
   cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FB_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (g_maps.size() > 4096) g_maps.clear();
+  g_maps.emplace(key, *out);
+  return FB_OK;
+}
+
+// Map of the packed queries [tokens, hq, d] bf16 as 3-D {d, hq, tokens}; the box is
+// 64 columns (the swizzle span) x g heads x bt tokens: a lean CTA's Q rows.
+fb_status q_map(const void* ptr, int tokens, int hq, int d, int g, int bt, CUtensorMap* out) {
+  std::memset(out, 0, sizeof(*out));
+  if (tokens <= 0) return FB_OK;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  char key[112];
+  snprintf(key, sizeof(key), "q%d:%p:%d:%d:%d:%d:%d", dev, ptr, tokens, hq, d, g, bt);
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return FB_OK;
+    }
+  }
+  EncodeTiledFn enc;
+  FB_TRY(get_encode(&enc));
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(hq), static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(hq) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(g), static_cast<cuuint32_t>(bt)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FB_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
@@ -397,6 +439,7 @@ fb_status fb_plan_query(const fb_problem* problem, int32_t call, fb_plan_info* o
   out->num_sms = sms;
   out->lean_reuse = pl.reuse ? 1 : 0;
   out->lean_smem_bytes = pl.reuse ? pl.reuse_smem : 0;
+  out->lean_early = pl.reuse && pl.reuse_early ? 1 : 0;
   return FB_OK;
 }
 
@@ -569,10 +612,14 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   prm.a_full = reinterpret_cast<__nv_bfloat16*>(a_full);
   prm.l_full = l_full;
   prm.decision_out = decision_out;
-  if (pl.reuse) {  // block K/V with 64-row boxes for the lean reuse path
+  if (pl.reuse && problem->total_q > 0 && problem->total_kv_in > 0) {
+    // block K/V with 64-row boxes and the Q box of a lean CTA
     FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, fb::kBN, &prm.tm_k_lean));
     FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, fb::kBN, &prm.tm_v_lean));
+    FB_TRY(q_map(q, problem->total_q, problem->num_heads_q, problem->head_dim, pl.g, pl.reuse_bt, &prm.tm_q_lean));
     prm.reuse_chunks = pl.reuse_chunks;
+    prm.reuse_bt = pl.reuse_bt;
+    prm.lean_early = pl.reuse_early ? 1 : 0;
     prm.lean = 1;
   }
   if (order_work) {

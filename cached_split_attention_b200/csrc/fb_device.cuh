@@ -115,6 +115,17 @@ __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* 
       : "memory");
 }
 
+// 3-D tiled bulk copy global -> shared (coordinates innermost first), default L2
+// policy, completion counted in bytes on `bar`.  No multicast.
+__device__ __forceinline__ void tma_load_3d_plain(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                                  int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Add `bytes` to the transaction count phase completion waits for (no arrival).
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");

@@ -101,7 +101,10 @@ struct alignas(64) Params {
   const uint32_t* out_skip;  // prefix tokens left out of J_out (bitmask; NULL: none)
   // lean reuse path (fb_reuse.cuh)
   CUtensorMap tm_k_lean, tm_v_lean;  // block K/V with 64-row boxes (the warp-MMA stage layout)
+  CUtensorMap tm_q_lean;             // Q as {d, hq, tokens}, box {64, g, reuse_bt}
   int reuse_chunks;  // 64-key chunks of the longest block
+  int reuse_bt;      // tokens of a lean CTA's Q box
+  int lean_early;    // 1: lean loads go out before the reuse decision (one-wave grids)
   int lean;          // 1: groups whose heads all reuse take the lean path
 };
 
@@ -120,38 +123,82 @@ __device__ __forceinline__ void prefetch_maps(const Params& p) {
     if (p.lean) {
       prefetch_tensormap(&p.tm_k_lean);
       prefetch_tensormap(&p.tm_v_lean);
+      prefetch_tensormap(&p.tm_q_lean);
     }
   }
 }
 
-// Reuse decision of (b, h); see fb_step in flashblock.h.
-__device__ __forceinline__ bool head_recompute(const Params& p, int b, int h) {
-  const int idx = b * p.hq + h;
-  if (!p.update_state) return p.head_mask ? (p.head_mask[idx] != 0) : true;
+// Reuse decision of (b, h) (true: recompute); see fb_step in flashblock.h.
+// Inputs of the decision of (b, h), loaded in one go (every load goes out before
+// any is tested: one memory round trip instead of a dependent chain) and tested by
+// decide(), so that a caller can do other work while they are in flight.
+struct DecisionIn {
+  int b, idx;
+  int mask, valid, reuse_in, n_upd, m_acc;
+  float cs;
+};
+__device__ __forceinline__ DecisionIn decision_load(const Params& p, int b, int h) {
+  DecisionIn d;
+  d.b = b;
+  d.idx = b * p.hq + h;
+  d.mask = d.valid = d.reuse_in = 1;
+  d.n_upd = d.m_acc = 0;
+  d.cs = 0.f;
+  if (!p.update_state) {
+    if (p.head_mask) d.mask = p.head_mask[d.idx];
+    return d;
+  }
+  if (p.flags & kForceRecompute) return d;
+  const bool tau = (p.flags & (kGateTau | kGateTauCum)) && p.n_updated;
+  d.valid = p.valid[d.idx];
+  d.reuse_in = p.head_reuse_in ? p.head_reuse_in[d.idx] : 1;
+  d.n_upd = tau ? p.n_updated[b] : 0;
+  d.m_acc = ((p.flags & kGateTauCum) && p.m_acc) ? p.m_acc[d.idx] : 0;
+  d.cs = (p.flags & kGateHead) ? p.cos[d.idx] : 0.f;
+  return d;
+}
+__device__ __forceinline__ bool decide(const Params& p, const DecisionIn& d) {
+  if (!p.update_state) return d.mask != 0;
   if (p.flags & kForceRecompute) return true;
-  if (!p.valid[idx]) return true;
+  if (!d.valid) return true;
   if (p.flags & kForceReuse) return false;
-  if (p.head_reuse_in) return p.head_reuse_in[idx] == 0;
+  if (p.head_reuse_in) return d.reuse_in == 0;
   bool reuse = true;
-  if (p.flags & kGateTau) reuse = reuse && (p.n_updated[b] < p.tau);
-  if (p.flags & kGateTauCum) reuse = reuse && (p.m_acc[idx] + p.n_updated[b] < p.tau);
-  if (p.flags & kGateHead) reuse = reuse && (p.cos[idx] > p.gamma);
+  if (p.flags & kGateTau) reuse = reuse && (d.n_upd < p.tau);
+  if (p.flags & kGateTauCum) reuse = reuse && (d.m_acc + d.n_upd < p.tau);
+  if (p.flags & kGateHead) reuse = reuse && (d.cs > p.gamma);
   return !reuse;
+}
+__device__ __forceinline__ bool head_recompute(const Params& p, int b, int h) {
+  return decide(p, decision_load(p, b, h));
+}
+
+// The state vote's loads, issued here and tested in state_vote (so that the
+// decision's loads go out beside them): at most 8 `valid` entries per thread.
+struct VoteLoads {
+  uint8_t e[8];  // the entries (1 where there is none)
+  bool all;      // every call updates state
+};
+__device__ __forceinline__ VoteLoads state_vote_load(const Params& p, int tid, int nthreads) {
+  VoteLoads v;
+  const int total = p.num_seqs * p.hq;
+  v.all = p.update_state && ((p.flags & kGateTauCum) || total > 8 * nthreads);
+  const bool load = p.update_state && !v.all;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int i = tid + k * nthreads;
+    v.e[k] = (load && i < total) ? p.valid[i] : uint8_t(1);
+  }
+  return v;
 }
 
 // Whether this call's last CTA has cache state to update: a head whose entry is
 // still empty (it becomes valid), or the cumulative count (kept on every call).
 // Every thread of the CTA calls it; the result is CTA-uniform through the vote.
-__device__ __forceinline__ bool state_vote(const Params& p, int tid, int nthreads) {
-  int need = 0;
-  if (p.update_state) {
-    const int total = p.num_seqs * p.hq;
-    if ((p.flags & kGateTauCum) || total > 8 * nthreads) {
-      need = 1;
-    } else {
-      for (int i = tid; i < total; i += nthreads) need |= p.valid[i] == 0;
-    }
-  }
+__device__ __forceinline__ bool state_vote(const VoteLoads& v) {
+  int need = v.all;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) need |= v.e[k] == 0;
   return __syncthreads_or(need) != 0;
 }
 
@@ -441,6 +488,7 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   float* cache_s = reinterpret_cast<float*>(smem + C::kOffCache);  // staged cache rows (kStageCache)
   __shared__ uint8_t s_rec[kMaxGroup];
   __shared__ int s_flag;
+  __shared__ __align__(8) uint64_t s_lean_bar[2];  // lean path: inputs, cached rows
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -473,15 +521,29 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   const int rows = ranges_ok ? n_q * g : 0;
   const int row0 = t * TR;
   const int nrows = max(0, min(TR, rows - row0));
-  int lean_r0 = 0, lean_nr = 0, lean_p = -1;  // this CTA's rows on the lean path, and its thread's position
-  if (p.lean && nrows > 0) {
-    lean_rows(nrows, split, S, lean_r0, lean_nr);
-    lean_p = lean_pos(p, q0, row0 + lean_r0, lean_nr, tid);
+  // Lean reuse path (fb_reuse.cuh): this CTA's rows of the group; in a one-wave
+  // grid their Q and the block K/V are loaded while the previous kernel finishes.
+  LeanRows lr{};
+  const LeanSmem<D> ls(smem, p.reuse_chunks, g, p.reuse_bt);
+  int lean_p = -1;  // block position of this thread's box token
+  if (p.lean && nrows > 0 && n_in <= p.reuse_chunks * kBN) {
+    int r0, nr;
+    lean_rows(nrows, split, S, r0, nr);
+    if (nr > 0) lr = lean_place(g, row0 + r0, nr);
   }
+  const bool lean_early = lr.nr > 0 && p.lean_early;
+  if (lr.nr > 0) lean_p = lean_pos(p, q0, lr, tid);
+  if (lean_early) lean_issue<D>(p, ls, s_lean_bar, hk, q0, in0, n_in, lr, tid);
   pdl_wait();
   pdl_trigger();
-  if (tid < g) s_rec[tid] = head_recompute(p, b, hk * g + tid) ? 1 : 0;
-  const bool need_state = state_vote(p, tid, C::kThreads);
+  // The decision's loads, the state vote's and the early cache rows go out
+  // together (the cache rows from warps 1.., after warp 0's decision loads).
+  const VoteLoads vote = state_vote_load(p, tid, C::kThreads);
+  DecisionIn din;
+  if (tid < g) din = decision_load(p, b, hk * g + tid);
+  if (lean_early) lean_fetch<D>(p, ls, s_lean_bar, hk, in0, n_in, lr, lean_p, tid);
+  if (tid < g) s_rec[tid] = decide(p, din) ? 1 : 0;
+  const bool need_state = state_vote(vote);
   bool any_rec = false;
   for (int j = 0; j < g; ++j) any_rec |= (s_rec[j] != 0);
 
@@ -508,11 +570,16 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
   if (p.decision_out && t == 0 && split == S - 1 && tid < g) p.decision_out[b * p.hq + hk * g + tid] = s_rec[tid];
   // A group whose heads all reuse takes the lean reuse path (its CTAs share the rows).
   const bool lean = p.lean && !any_rec && active;
+  if (!lean && lean_early) lean_drain(s_lean_bar, tid);
   if (lean) {
     if (n_in > p.reuse_chunks * kBN) {
       if (tid == 0) record_status(kDevBadIndex);
-    } else if (lean_nr > 0) {
-      lean_reuse<D>(p, smem, b, hk, q0, in0, n_in, row0 + lean_r0, lean_nr, lean_p, tid, C::kThreads);
+    } else if (lr.nr > 0) {
+      if (!lean_early) {
+        lean_issue<D>(p, ls, s_lean_bar, hk, q0, in0, n_in, lr, tid);
+        lean_fetch<D>(p, ls, s_lean_bar, hk, in0, n_in, lr, lean_p, tid);
+      }
+      lean_finish<D>(p, ls, s_lean_bar, lr, q0, hk, n_in, tid, C::kThreads);
     }
   } else if (active && (has_in || has_out || cluster_mode)) {
     // -------------------------------------------------------- Q rows first
@@ -633,7 +700,7 @@ __global__ void __launch_bounds__(Cfg<D, WM, WN, STAGES>::kThreads, 1) attn_kern
     auto skip_of = [&](int c) -> uint64_t {
       if (!p.out_skip || c < nA || c >= n_local) return 0ull;
       uint64_t w = skip_bits64(p.out_skip, p.total_out, out0 + (pa + c - nA) * kBN + wn * KW);
-      if (KW < 64) w &= (1ull << KW) - 1ull;
+      if constexpr (KW < 64) w &= (1ull << (KW % 64)) - 1ull;
       return w;
     };
     // One segment of chunks [c0, c1) of the local sequence.

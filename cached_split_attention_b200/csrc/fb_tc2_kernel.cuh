@@ -98,8 +98,9 @@ __global__ void __launch_bounds__(tc2::kThreads, 1) tc2_attn_kernel(const __grid
   const int n_out = p.cu_out[b + 1] - out0;
   const int in0 = p.cu_in[b];
   const int n_in = p.cu_in[b + 1] - in0;
+  const VoteLoads vote = state_vote_load(p, tid, kThreads);
   if (tid == 0) s_rec0 = head_recompute(p, b, h) ? 1 : 0;
-  const bool need_state = state_vote(p, tid, kThreads);
+  const bool need_state = state_vote(vote);
   const bool rec = s_rec0 != 0;
   const bool ranges_ok = q0 >= 0 && n_q >= 0 && q0 + n_q <= p.total_q && out0 >= 0 && n_out >= 0 &&
                          out0 + n_out <= p.total_out && in0 >= 0 && n_in >= 0 && in0 + n_in <= p.total_in &&

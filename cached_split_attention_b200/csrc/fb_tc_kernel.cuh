@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   float* part_in = reinterpret_cast<float*>(smem + kOffPartIn);
   __shared__ uint8_t s_rec[kMaxGroup];
   __shared__ int s_flag;
+  __shared__ __align__(8) uint64_t s_lean_bar[2];  // lean path: inputs, cached rows
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -167,15 +168,28 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   if (!ranges_ok && tid == 0 && t == 0 && split == 0) record_status(kDevBadIndex);
   const int rows = ranges_ok ? n_q * g : 0;
   const int nrows = max(0, min(kM, rows - row0));
-  int lean_r0 = 0, lean_nr = 0, lean_p = -1;  // this CTA's rows on the lean path, and its thread's position
-  if (p.lean && nrows > 0) {
-    lean_rows(nrows, split, S, lean_r0, lean_nr);
-    lean_p = lean_pos(p, q0, row0 + lean_r0, lean_nr, tid);
+  // Lean reuse path (see attn_kernel).
+  LeanRows lr{};
+  const LeanSmem<kD> ls(smem, p.reuse_chunks, g, p.reuse_bt);
+  int lean_p = -1;  // block position of this thread's box token
+  if (p.lean && nrows > 0 && n_in <= p.reuse_chunks * kBN) {
+    int r0, nr;
+    lean_rows(nrows, split, S, r0, nr);
+    if (nr > 0) lr = lean_place(g, row0 + r0, nr);
   }
+  const bool lean_early = lr.nr > 0 && p.lean_early;
+  if (lr.nr > 0) lean_p = lean_pos(p, q0, lr, tid);
+  if (lean_early) lean_issue<kD>(p, ls, s_lean_bar, hk, q0, in0, n_in, lr, tid);
   pdl_wait();
   pdl_trigger();
-  if (tid < g) s_rec[tid] = head_recompute(p, b, hk * g + tid) ? 1 : 0;
-  const bool need_state = state_vote(p, tid, kThreads);
+  // The decision's loads, the state vote's and the early cache rows go out
+  // together (the cache rows from warps 1.., after warp 0's decision loads).
+  const VoteLoads vote = state_vote_load(p, tid, kThreads);
+  DecisionIn din;
+  if (tid < g) din = decision_load(p, b, hk * g + tid);
+  if (lean_early) lean_fetch<kD>(p, ls, s_lean_bar, hk, in0, n_in, lr, lean_p, tid);
+  if (tid < g) s_rec[tid] = decide(p, din) ? 1 : 0;
+  const bool need_state = state_vote(vote);
   bool any_rec = false;
   for (int j = 0; j < g; ++j) any_rec |= (s_rec[j] != 0);
 
@@ -197,11 +211,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   if (p.decision_out && t == 0 && split == S - 1 && tid < g) p.decision_out[b * p.hq + hk * g + tid] = s_rec[tid];
   // A group whose heads all reuse takes the lean reuse path (its CTAs share the rows).
   const bool lean = p.lean && !any_rec && active;
+  if (!lean && lean_early) lean_drain(s_lean_bar, tid);
   if (lean) {
     if (n_in > p.reuse_chunks * kBN) {
       if (tid == 0) record_status(kDevBadIndex);
-    } else if (lean_nr > 0) {
-      lean_reuse<kD>(p, smem, b, hk, q0, in0, n_in, row0 + lean_r0, lean_nr, lean_p, tid, kThreads);
+    } else if (lr.nr > 0) {
+      if (!lean_early) {
+        lean_issue<kD>(p, ls, s_lean_bar, hk, q0, in0, n_in, lr, tid);
+        lean_fetch<kD>(p, ls, s_lean_bar, hk, in0, n_in, lr, lean_p, tid);
+      }
+      lean_finish<kD>(p, ls, s_lean_bar, lr, q0, hk, n_in, tid, kThreads);
     }
   } else if (active && (has_in || has_out || cluster_mode)) {
     // -------------------------------------------------------- Q rows (before the K/V stream)
@@ -397,7 +416,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
         }
       } else {
         // ---------------------------------------------------- rows: softmax
-        const int r = tid;
         float m = kNegInf, l = 0.f;
         bool ok = true;
         // skip-mask bits of a prefix chunk's 128 keys, loaded one chunk ahead

@@ -86,11 +86,17 @@ typedef enum fb_status {
  * out_splits: number of key splits of the prefix pass; 0 lets the library choose.
  * Ordering: the attention calls read the index arrays (cu_seqlens_*, q_rows) before they
  *   wait for the previous kernel of the stream to finish, so that these loads overlap its
- *   tail.  A kernel that precedes such a call on its stream and lets its dependents launch
- *   early (programmatic dependent launch, griddepcontrol.launch_dependents) must not write
- *   them; ordinary kernels and copies are waited for as usual.  The library's own kernels
- *   that write index arrays (fb_sparse_layout, fb_prefix_append) do not launch dependents
- *   early.  Everything else (Q/K/V, the cache, kv_out_skip) is read after the wait.
+ *   tail; fb_step with early lean loads (fb_plan_info.lean_early) also reads its block
+ *   inputs q, k_in and v_in there.  A kernel that precedes such a call on its stream
+ *   and lets its dependents launch early (programmatic dependent launch,
+ *   griddepcontrol.launch_dependents) must not write any of them; ordinary kernels
+ *   and copies are waited for as usual.  The library's own
+ *   kernels that write index arrays or block K/V (fb_sparse_layout, fb_prefix_append) do
+ *   not launch dependents early, and none writes q.  The attention kernels themselves
+ *   do launch their dependents early, so an output of one call (a_full, l_full, the
+ *   cache) must not be read as q, k_in or v_in by the next attention call on the stream
+ *   without an ordinary kernel or copy in between.  Everything else (the prefix K/V, the
+ *   cache, kv_out_skip) is read after the wait.
  * kv_out_skip: NULL, or a bitmask over the prefix tokens (device, uint32 words, at least
  *   ceil(total_kv_out / 32) of them): bit t (bit t % 32 of word t / 32) set leaves prefix
  *   token t -- row t of k_out / v_out -- out of J_out.  The sparse-residual layout
@@ -175,6 +181,8 @@ typedef struct fb_plan_info {
    * one round of loads. */
   int32_t lean_reuse;      /* 1 when the call has the lean path                     */
   int32_t lean_smem_bytes; /* shared memory it uses per CTA at most (of smem_bytes) */
+  int32_t lean_early;      /* 1 when its loads start before the reuse decision is known
+                              (the grid is resident in one wave); see Ordering       */
 } fb_plan_info;
 
 /*

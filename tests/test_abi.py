@@ -191,7 +191,9 @@ def test_plan_query_matches_the_bench_kernel_map():
 def test_plan_query_lean_reuse_path():
     """The lean reuse path: planned for fused steps of blocks of at most 128 keys
     (every bench workload but the 1560-token video block), never for the unfused
-    passes, and only when the kernel's shared memory holds what it needs."""
+    passes, and only when the kernel's shared memory holds what it needs.  Its loads
+    start before the reuse decision only when the whole grid is resident at once
+    (one CTA per SM here: at most num_sms CTAs), so not for the 192-CTA varlen grid."""
     _built()
     from cached_split_attention_b200 import binding as B
     for name, p in _shape_problems().items():
@@ -200,8 +202,15 @@ def test_plan_query_lean_reuse_path():
         assert step["lean_reuse"] == (0 if name == "video" else 1), (name, step)
         if step["lean_reuse"]:
             assert 0 < step["lean_smem_bytes"] <= step["smem_bytes"], (name, step)
+            one_wave = step["ctas"] <= step["num_sms"] * max(1, 233472 // (step["smem_bytes"] + 1024))
+            assert step["lean_early"] == int(one_wave), (name, step)
+        else:
+            assert step["lean_early"] == 0
         for call in (B.CALL_OUT, B.CALL_IN):
-            assert B.plan_query(dp, call)["lean_reuse"] == 0
+            info = B.plan_query(dp, call)
+            assert info["lean_reuse"] == 0 and info["lean_early"] == 0
+    early = {n: B.plan_query(B.DeviceProblem(p, "cpu"))["lean_early"] for n, p in _shape_problems().items()}
+    assert early["long_context_gqa"] == 1 and early["dllm_layer"] == 1 and early["varlen_branches"] == 0
 
 
 def test_plan_query_rejects_bad_arguments():
