@@ -875,6 +875,18 @@ def _rows_sparse(torch, B, device, flush, flush_out, reps, clocks, out_rows, hbm
             launches += reps
             del g
     launches += reps
+    # the layout where it runs: on the stream in front of the sparse recompute call
+    # that reads what it writes (the difference is its marginal cost there)
+    prm_rec = B.params(0, 0.0, W.FORCE_RECOMPUTE)
+
+    def layout_then_step(st_):
+        layout(st_)
+        sp.step(prm_rec, st_)
+
+    g_both = _graph_of(torch, layout_then_step)
+    t_both = _cold_us(torch, g_both, flush, flush_out, reps, clocks)
+    launches += 2 * reps
+    del g_both
     lb = sparse_layout_bytes(p, total_sel)
     ach = lb / float(np.median(t_lay)) / 1e3
 
@@ -892,7 +904,14 @@ def _rows_sparse(torch, B, device, flush, flush_out, reps, clocks, out_rows, hbm
                      f"{total_sel // p.num_seqs} of {p.max_kv_out} keys",
         "layout": dict(_stats(t_lay), call="fb_sparse_layout", algorithmic_bytes=lb,
                        roofline={"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
-                                 "frac": round(ach / hbm_peak, 4), "peak_source": peak_src}),
+                                 "frac": round(ach / hbm_peak, 4), "peak_source": peak_src},
+                       timing="alone: one call per graph replay after an L2 flush"),
+        "layout_then_recompute": dict(
+            _stats(t_both), calls="fb_sparse_layout then fb_step (sparse, recompute) in one graph",
+            layout_marginal_us=round(float(np.median(t_both)) - float(np.median(timed[("sparse", "recompute")])), 3),
+            layout_marginal_frac_of_dense_recompute=round(
+                (float(np.median(t_both)) - float(np.median(timed[("sparse", "recompute")]))) /
+                float(np.median(timed[("dense", "recompute")])), 4)),
         "step_sparse": {"recompute_call_us": arm("sparse", "recompute", 1.0),
                         "reuse_call_us": arm("sparse", "reuse", 0.0)},
         "step_dense": {"recompute_call_us": arm("dense", "recompute", 1.0),

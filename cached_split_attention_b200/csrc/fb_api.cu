@@ -702,11 +702,6 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
   if (kv_out_skip && (reinterpret_cast<uintptr_t>(kv_out_skip) & 3u))
     return fail(FB_ERR_INVALID_ARG, "kv_out_skip is not 4-byte aligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t words = (static_cast<size_t>(problem->total_kv_out) + 31) / 32;
-  if (words) {
-    cudaError_t e = cudaMemsetAsync(kv_out_skip, 0, words * sizeof(uint32_t), st);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(kv_out_skip)");
-  }
   fb::SparseParams sp{problem->num_seqs, problem->num_heads_kv, problem->head_dim, problem->total_kv_out,
                       problem->total_kv_in, total_sel, problem->cu_seqlens_kv_out, problem->cu_seqlens_kv_in, cu_sel,
                       sel_idx, reinterpret_cast<const __nv_bfloat16*>(k_out),

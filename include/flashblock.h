@@ -305,7 +305,9 @@ fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* ca
  * total_sel (host) = cu_sel[num_seqs].  Outputs (device, caller-owned):
  *   k_ext, v_ext [total_kv_in + total_sel, H_kv, d] (THD bf16): J_in' of every sequence;
  *   kv_out_skip [ceil(total_kv_out / 32)] uint32: the bitmask of the selected prefix
- *     tokens (bit t of the global prefix row t), cleared and set by this call;
+ *     tokens (bit t of the global prefix row t); this call writes the bits of every
+ *     sequence's prefix tokens (cleared, then the selected ones set) and leaves bits
+ *     past total_kv_out as they are;
  *   cu_seqlens_kv_in_ext = cu_seqlens_kv_in + cu_sel ([num_seqs+1]; may be NULL).
  * The residual prefix is not copied: J_out' is the prefix (k_out, v_out,
  * cu_seqlens_kv_out unchanged) with kv_out_skip set in the problem, which every prefix
@@ -314,9 +316,12 @@ fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* ca
  * total_kv_in + total_sel rows caches the residual and recomputes the selected keys every
  * step; with a fresh cache the result is full attention over prefix and block.  The
  * selection is fixed for a block (a new one changes the residual: refill the cache).
- * The pass moves the block rows and the selected rows only.  A selection that is not
- * increasing or out of range records FB_ERR_INVALID_ARG on the device (fb_device_status);
- * that sequence is skipped.  At most 65535 sequences per call (FB_ERR_UNSUPPORTED beyond).
+ * The pass moves the block rows and the selected rows only, in one kernel.  A selection
+ * that is not increasing or out of range records FB_ERR_INVALID_ARG on the device
+ * (fb_device_status); that sequence's skip bits are left cleared and its
+ * cu_seqlens_kv_in_ext entry unwritten, and its J_in' rows are unspecified (the
+ * selected rows next to a bad entry are not written).  A sequence whose offsets are
+ * inconsistent is not touched at all.  At most 65535 sequences per call (FB_ERR_UNSUPPORTED beyond).
  */
 fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, const int32_t* sel_idx,
                            int32_t total_sel, const fb_bf16* k_out, const fb_bf16* v_out, const fb_bf16* k_in,
