@@ -96,6 +96,7 @@ struct Plan {
   int d = 0, g = 0, wm = 0, tr = 0, tiles = 0, n_groups = 0, splits = 1, threads = 0, smem = 0;
   bool tc = false;   // tensor-core kernel (tcgen05): head_dim 128, more than 64 rows per group
   bool tc2 = false;  // two-tile tensor-core kernel: fused step, MHA, at least 256 rows per head
+  bool tc_split = false;  // tensor-core kernel with two threads per tile row (grids of more than one wave)
   int bn = fb::kBN;  // keys per pipeline chunk (TMA box rows)
   size_t off_grid_ctr = 0, off_cos = 0, off_order = 0, bytes = 0;
   int order_items = 0;  // work items of the two-tile kernel (0: the problem never takes it)
@@ -171,7 +172,7 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = fals
     pl.tr = 2 * fb::tc2::kM;
     pl.bn = fb::tc2::kN;
   } else if (pl.tc) {
-    pl.threads = fb::tc::kThreads;
+    pl.threads = fb::tc::threads_for(1);
     pl.smem = fb::tc::kSmem;
     pl.tr = fb::tc::kM;
     pl.bn = fb::tc::kN;
@@ -200,6 +201,17 @@ Plan make_plan(const fb_problem* p, int num_sms, bool in_only, bool fused = fals
     splits = std::max(1, std::min({splits, fb::kMaxSplits, chunks}));
   }
   pl.splits = splits;
+  // More CTAs than one wave holds (the varlen branches): the later CTAs run with the
+  // HBM less loaded, where one softmax thread per row bounds the stream; two threads
+  // per row (twice the softmax warps) suit them.  A full single wave is bound by HBM,
+  // and there the extra per-chunk exchange of the two halves costs a little.
+  if (pl.tc && !pl.tc2) {
+    const int per_sm = std::max(1, std::min(233472 / (pl.smem + 1024), 2048 / pl.threads));
+    if (static_cast<long>(pl.n_groups) * pl.splits > static_cast<long>(num_sms) * per_sm) {
+      pl.tc_split = true;
+      pl.threads = fb::tc::threads_for(2);
+    }
+  }
   // Lean reuse path: blocks of up to 128 keys, when the kernel's shared memory
   // holds the block K/V and a tile of rows with their cache entries.
   if (fused && !pl.tc2 && p->max_kv_in > 0 && p->max_kv_in <= fb::reuse::kMaxKeys && rows > 0) {
@@ -331,13 +343,14 @@ fb_status launch_attn(const Plan& pl, fb::Params& prm, cudaStream_t stream) {
   const int n_ctas = pl.n_groups * pl.splits;
   if (n_ctas <= 0) return FB_OK;
   void* fn = pl.tc2  ? reinterpret_cast<void*>(&fb::tc2_attn_kernel)
-             : pl.tc ? reinterpret_cast<void*>(&fb::tc_attn_kernel)
+             : pl.tc ? (pl.tc_split ? reinterpret_cast<void*>(&fb::tc_attn_kernel<2>)
+                                    : reinterpret_cast<void*>(&fb::tc_attn_kernel<1>))
                      : shape_for(pl.d, pl.wm).fn;
   static std::mutex mu;
-  static bool attr_done[4][9] = {};
+  static bool attr_done[5][9] = {};
   {
     std::lock_guard<std::mutex> lk(mu);
-    bool& done = attr_done[pl.tc2 ? 3 : pl.tc ? 2 : (pl.d == 128)][pl.wm];
+    bool& done = attr_done[pl.tc2 ? 3 : pl.tc ? (pl.tc_split ? 4 : 2) : (pl.d == 128)][pl.wm];
     if (!done) {
       cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");

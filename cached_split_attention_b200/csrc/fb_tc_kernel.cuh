@@ -10,20 +10,31 @@
 // log-space merge through distributed shared memory.  What changes is the inner
 // loop, per 128-key chunk:
 //
-//   warp 4 (one thread)  TMA: K chunk -> ring of 3, V chunk -> ring of 3
-//   warp 5 (one thread)  S = Q K^T   (tcgen05.mma, M=128 N=128 K=128, fp32 in TMEM,
-//                                     two S buffers so the next chunk's S overlaps
-//                                     the softmax of this one)
-//                        O += P V    (tcgen05.mma with A = P read from TMEM, O in
-//                                     TMEM; one O accumulator per segment)
-//   warps 0-3            one thread per tile row (= TMEM lane): load the S row,
-//                        mask, running max in base 2, P = 2^(s - m) rounded to bf16
-//                        and stored back over the S row it came from; O is rescaled
-//                        in TMEM only when the running max grows by more than 2^8
-//                        (the stored max may lag: exact, since O and l always share
-//                        the same reference).  Three of every eight 2^x go through a
-//                        cubic on the FMA pipe instead of the MUFU unit, whose
-//                        throughput otherwise bounds the softmax.
+//   warp 4R (one thread)    TMA: K chunk -> ring of 3, V chunk -> ring of 3
+//   warp 4R+1 (one thread)  S = Q K^T   (tcgen05.mma, M=128 N=128 K=128, fp32 in
+//                                        TMEM, two S buffers so the next chunk's S
+//                                        overlaps the softmax of this one)
+//                           O += P V    (tcgen05.mma with A = P read from TMEM, O in
+//                                        TMEM; one O accumulator per segment)
+//   warps 0 .. 4R-1         R threads per tile row (= TMEM lane): warp w takes keys
+//                           128 (w / 4) / R .. of the rows of lane quarter w % 4.
+//                           Each loads its share of the S row and masks it, runs the
+//                           max in base 2, P = 2^(s - m) rounded to bf16 and stored
+//                           back over S columns already read, and its sum.  O is
+//                           rescaled in TMEM only when the running max grows by more
+//                           than 2^8 (the stored max may lag: exact, since O and l
+//                           always share the same reference).  Three of every eight
+//                           2^x go through a cubic on the FMA pipe instead of the
+//                           MUFU unit.
+//
+// R = 1 in a grid that one wave holds, where the stream is bound by HBM.  R = 2
+// (the host plan's choice for more CTAs than one wave, e.g. the varlen branches,
+// whose later CTAs run with the HBM less loaded): one softmax thread per row is
+// bound by its own latencies, and two softmax warps per SM sub-partition fill each
+// other's stalls.  The two halves of a row swap their maxima through shared memory
+// each chunk (bounded mbarrier handshakes) and add their sums at the end.  R = 2 took
+// the varlen branches' recompute call from 82.2 to 73.6 us; on the long-context GQA
+// batch (one wave, HBM-bound) it cost 1 % per call.
 //
 // The MMA thread issues S(c) after P V(c-2) and P V(c) after S(c+1); the tensor
 // core runs them in issue order, so S(c+2) never overwrites P(c) before P V(c) has
@@ -48,7 +59,9 @@ namespace tc {
 constexpr int kD = 128;
 constexpr int kM = 128;           // tile rows = TMEM lanes
 constexpr int kN = 128;           // keys per chunk
-constexpr int kThreads = 192;     // warps 0-3 rows, warp 4 TMA, warp 5 MMA
+// Threads of a CTA with R threads per tile row: 4 R row warps, then the TMA warp
+// and the MMA warp.
+constexpr int threads_for(int row_threads) { return 128 * row_threads + 64; }
 constexpr int kHalf = kN * 128;   // 64 columns (128 bytes) x 128 rows: 16 KB
 constexpr int kTile = 2 * kHalf;  // 128 x 128 bf16: 32 KB
 constexpr int kStages = 3;        // K and V rings
@@ -117,9 +130,13 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 }  // namespace tc
 
-__global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_constant__ Params p) {
+template <int kRowThreads>
+__global__ void __launch_bounds__(tc::threads_for(kRowThreads), 1) tc_attn_kernel(const __grid_constant__ Params p) {
   prefetch_maps(p);
   using namespace tc;
+  constexpr int kThreads = threads_for(kRowThreads);
+  constexpr int kTmaWarp = 4 * kRowThreads;  // warps 0 .. 4R-1 hold the rows
+  constexpr int kMmaWarp = kTmaWarp + 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -139,6 +156,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
   __shared__ uint8_t s_rec[kMaxGroup];
   __shared__ int s_flag;
   __shared__ __align__(8) uint64_t s_lean_bar[2];  // lean path: inputs, cached rows
+  // the two softmax warps of a row quarter swap per-row values (the halves' maxima
+  // of a chunk, their sums at the end) through s_xv; s_xch: both written, s_xrd:
+  // both read (so that a slot is rewritten only after the other warp has read it)
+  __shared__ __align__(8) uint64_t s_xch[4], s_xrd[4];
+  __shared__ float s_xv[kRowThreads][kRowThreads == 2 ? kM : 1];
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -269,7 +291,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
       tma_load_2d(dst + kHalf, map, bar, hk * kD + 64, y, pol);
     };
     // The TMA thread initialises the barriers and starts the stream at once.
-    if (warp == 4 && lane == 0) {
+    if (warp == kTmaWarp && lane == 0) {
       for (int i = 0; i < kStages; ++i) {
         mbar_init(&k_full[i], 1);
         mbar_init(&k_empty[i], 1);
@@ -278,7 +300,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
       }
       mbar_init(&s_full[0], 1);
       mbar_init(&s_full[1], 1);
-      mbar_init(p_full, kM / 32);  // one arrival per row warp
+      mbar_init(p_full, kRowThreads * kM / 32);  // one arrival per row warp
+      for (int i = 0; i < 4; ++i) {  // two threads per row: the two warps of a lane quarter
+        mbar_init(&s_xch[i], 2);   // both values written
+        mbar_init(&s_xrd[i], 2);   // both read
+      }
       mbar_init(pv_done, 1);
       mbar_init(drain, 1);
       *s_abort = 0;
@@ -288,7 +314,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
         load(c, true);
       }
     }
-    if (warp == 5 && n_local > 0) {
+    if (warp == kMmaWarp && n_local > 0) {
       tmem_alloc(s_tmem, kTmemCols);
       tmem_relinquish();
     }
@@ -323,9 +349,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
     }
 
     float m_in = kNegInf, l_in = 0.f, m_out = kNegInf, l_out = 0.f;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);  // rows warps only
+    // rows warps only: warp w holds TMEM lanes 32 (w % 4) .. + 31, keys 64 (w / 4) .. + 63
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     if (n_local > 0) {
-      if (warp == 4) {
+      if (warp == kTmaWarp) {
         // ---------------------------------------------------- TMA producer
         if (lane == 0) {
           int issued_k = min(kStages, n_local), issued_v = issued_k;
@@ -355,7 +382,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
               if (!mbar_wait(&v_full[c % kStages], (c / kStages) & 1)) record_status(kDevTimeout);
           }
         }
-      } else if (warp == 5) {
+      } else if (warp == kMmaWarp) {
         // ---------------------------------------------------- MMA issuer
         if (lane == 0) {
           const uint32_t q_a = smem_u32(smem + kOffQ);
@@ -414,8 +441,192 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
           umma_commit(drain);  // every MMA issued has finished before the CTA moves on
           if (!mbar_wait(drain, 0)) record_status(kDevTimeout);
         }
-      } else {
+      } else if constexpr (kRowThreads == 2) {
         // ---------------------------------------------------- rows: softmax
+        // Two threads per row: warp w takes keys 64 h .. 64 h + 63 (h = w / 4) of
+        // the rows of TMEM lane quarter w % 4, so that each SM sub-partition runs
+        // two softmax warps that fill each other's stalls.  The halves share the
+        // running max of the row (one exchange per chunk) and keep their own sums.
+        const int h = warp >> 2;
+        const int qr = warp & 3;
+        const int r = qr * 32 + lane;  // the row = TMEM lane
+        float m = kNegInf, l = 0.f;
+        bool ok = true;
+        int round = 0;  // exchanges made with the other half's warp
+        // this half's value of the row for the other half's, both bounded waits
+        auto exchange = [&](float v) -> float {
+          if (round > 0 && !__all_sync(0xffffffffu, mbar_wait(&s_xrd[qr], (round - 1) & 1))) ok = false;
+          s_xv[h][r] = v;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_xch[qr]);
+          if (!__all_sync(0xffffffffu, mbar_wait(&s_xch[qr], round & 1))) ok = false;
+          tc_fence_after();
+          const float o = s_xv[h ^ 1][r];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_xrd[qr]);
+          ++round;
+          return o;
+        };
+        // skip-mask bits of this half's 64 keys of a prefix chunk, loaded one chunk ahead
+        auto skip_of = [&](int c) -> uint64_t {
+          if (!p.out_skip || c < nA || c >= n_local) return 0ull;
+          return skip_bits64(p.out_skip, p.total_out, out0 + (pa + c - nA) * kN + 64 * h);
+        };
+        uint64_t skip_next = skip_of(0);
+        for (int c = 0; c < n_local; ++c) {
+          const uint64_t skip = skip_next;  // bit k: key 64 h + k of the chunk left out
+          skip_next = skip_of(c + 1);
+          if (c == nA && c > 0) {  // block segment done; the prefix segment starts
+            m_in = m;
+            l_in = l;
+            m = kNegInf;
+            l = 0.f;
+          }
+          const uint32_t sp = lane_base + kColS + (c & 1) * kN;  // S(c), then P(c)
+          const bool seg_in = c < nA;
+          const int key0 = seg_in ? c * kN : (pa + c - nA) * kN;
+          const int valid = min(kN, (seg_in ? n_in : n_out) - key0) - 64 * h;  // of this half's keys
+          const bool first = c == 0 || c == nA;
+          if (!__all_sync(0xffffffffu, mbar_wait(&s_full[c & 1], (c >> 1) & 1))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t sv[2][32];
+          tmem_ld32(sp + 64 * h, sv[0]);
+          tmem_ld32(sp + 64 * h + 32, sv[1]);
+          tmem_wait_ld();
+          reg_fence32(sv[0]);
+          reg_fence32(sv[1]);
+          // Keys past the segment's end, and prefix keys the skip mask leaves out,
+          // get -inf; the row max of the raw scores (the scale is positive, so it
+          // commutes with the max) in four chains of 3-input maxima.
+          if (valid < 64 || skip) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (32 * i + k >= valid || ((skip >> (32 * i + k)) & 1ull)) sv[i][k] = __float_as_uint(kNegInf);
+            }
+          }
+          float mxa[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 2)
+              mxa[(k >> 1) & 3] = max3(mxa[(k >> 1) & 3], __uint_as_float(sv[i][k]), __uint_as_float(sv[i][k + 1]));
+          }
+          const float mxh = fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3]));
+          // Both halves have read their scores once the exchange is through, so P
+          // may be written over S below (half 1's P lands on half 0's S columns).
+          const float mxo = exchange(mxh);
+          if (!ok) break;
+          const float mx = fmaxf(mxh, mxo) * p.scale_log2;
+          const float m_new = fmaxf(m, mx);
+          float alpha = 1.f;
+          bool resc = false;
+          if (first) {
+            m = m_new;
+          } else if (m_new > m + kRescaleSlack) {
+            alpha = ex2(m - m_new);
+            m = m_new;
+            resc = true;
+          }
+          const float nm = m == kNegInf ? 0.f : -m;
+          // P = 2^(s * scale - m), rounded to bf16 for the P V product; paired fp32
+          // arithmetic, pairs 8a+0..2 of every eight by the cubic, the rest by MUFU;
+          // the half-row sum in eight chains (four paired accumulators).
+          uint32_t pk[32];  // packed bf16 pairs: keys 64 h + 2j, 64 h + 2j + 1 in column 32 h + j
+          uint64_t rsa[4];
+#pragma unroll
+          for (int a2 = 0; a2 < 4; ++a2) rsa[a2] = 0ull;
+          const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+          const uint64_t nm2 = f2_pack(nm, nm);
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+              const uint64_t x = ffma2(f2_pack(__uint_as_float(sv[i][k]), __uint_as_float(sv[i][k + 1])), scale2, nm2);
+              float p0, p1;
+              if (((k >> 1) & 7) < 3) {
+                exp2_poly2(x, p0, p1);
+              } else {
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              rsa[(k >> 1) & 3] = fadd2(rsa[(k >> 1) & 3], f2_pack(p0, p1));
+              pk[16 * i + k / 2] = pack_bf16x2(p0, p1);
+            }
+          }
+          float r0, r1, r2, r3, r4, r5, r6, r7;
+          f2_unpack(rsa[0], r0, r1);
+          f2_unpack(rsa[1], r2, r3);
+          f2_unpack(rsa[2], r4, r5);
+          f2_unpack(rsa[3], r6, r7);
+          const float rs = ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
+          l = l * alpha + rs;
+          // P V(c-1) must be finished before O is rescaled; otherwise the wait only
+          // keeps the rows in step with the MMA thread (one wait per chunk, before
+          // P(c) is published, so the phase waited for is never overtaken).  The
+          // decision is the same in both halves (same maxima), each rescales its
+          // half of O.
+          const bool rescale = __any_sync(0xffffffffu, resc);
+          bool waited = c == 0;
+          if (rescale) {
+            if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (c - 1) & 1))) {
+              ok = false;
+              break;
+            }
+            waited = true;
+            tc_fence_after();
+            const uint32_t oc = lane_base + (seg_in ? kColIn : kColOut) + 64 * h;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              uint32_t o[32];
+              tmem_ld32(oc + 32 * i, o);
+              tmem_wait_ld();
+              reg_fence32(o);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+              tmem_st32(oc + 32 * i, o);
+            }
+          }
+          // P(c) over S(c) columns whose scores both halves have read (see above)
+          tmem_st32(sp + 32 * h, pk);
+          tmem_wait_st();
+          if (!waited) {
+            if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (c - 1) & 1))) {
+              ok = false;
+              break;
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full);
+        }
+        if (ok && !__all_sync(0xffffffffu, mbar_wait(pv_done, (n_local - 1) & 1))) ok = false;
+        if (!ok) {
+          if (lane == 0) record_status(kDevTimeout);
+          *s_abort = 1;
+        }
+        tc_fence_after();
+        if (nB > 0) {
+          m_out = m;
+          l_out = l;
+        } else {
+          m_in = m;
+          l_in = l;
+        }
+        // the rows' sums: this half's and the other half's
+        if (ok) {
+          l_in += exchange(l_in);
+          l_out += exchange(l_out);
+        }
+      } else {
+        // ---------------------------------------------------- rows: softmax, one thread per row
         float m = kNegInf, l = 0.f;
         bool ok = true;
         // skip-mask bits of a prefix chunk's 128 keys, loaded one chunk ahead
@@ -577,15 +788,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
     tc_fence_after();
 
     // -------------------------------------------------------- partials -> shared memory
-    if (warp < 4 && n_local > 0) {
-      const int r = tid;
+    if (warp < 4 * kRowThreads && n_local > 0) {  // a row's threads: their shares of the columns
+      constexpr int kCols = kD / kRowThreads;
+      const int r = (warp & 3) * 32 + lane;
+      const int h = warp >> 2;
       auto store = [&](float* part, uint32_t col, float mm, float ll) {
         const float inv = ll > 0.f ? 1.f / ll : 0.f;
-        float* row = part + r * kPStride;
+        float* row = part + r * kPStride + kCols * h;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kCols / 32; ++i) {
           uint32_t o[32];
-          tmem_ld32(lane_base + col + 32 * i, o);
+          tmem_ld32(lane_base + col + kCols * h + 32 * i, o);
           tmem_wait_ld();
           reg_fence32(o);
 #pragma unroll
@@ -594,7 +807,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
                 make_float4(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv,
                             __uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
         }
-        part[kPartL + r] = ll > 0.f ? (mm + log2f(ll)) * kLn2 : kNegInf;
+        if (h == 0) part[kPartL + r] = ll > 0.f ? (mm + log2f(ll)) * kLn2 : kNegInf;
       };
       if (nA > 0) store(part_in, kColIn, m_in, l_in);
       if (nB > 0) store(part_out, kColOut, m_out, l_out);
@@ -605,7 +818,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1) tc_attn_kernel(const __grid_c
     } else {
       __syncthreads();
     }
-    if (warp == 5 && n_local > 0) {
+    if (warp == kMmaWarp && n_local > 0) {
       tc_fence_after();
       tmem_dealloc(tmem, kTmemCols);
     }

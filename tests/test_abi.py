@@ -213,6 +213,20 @@ def test_plan_query_lean_reuse_path():
     assert early["long_context_gqa"] == 1 and early["dllm_layer"] == 1 and early["varlen_branches"] == 0
 
 
+def test_plan_query_tensor_core_threads_per_row():
+    """The tensor-core kernel runs one softmax thread per tile row in a grid that one
+    wave holds (192 threads) and two per row beyond it (320 threads): the long-context
+    GQA batch is one wave of 128 CTAs, the varlen branches 192 CTAs."""
+    _built()
+    from cached_split_attention_b200 import binding as B
+    probs = _shape_problems()
+    gqa = B.plan_query(B.DeviceProblem(probs["long_context_gqa"], "cpu"))
+    var = B.plan_query(B.DeviceProblem(probs["varlen_branches"], "cpu"))
+    assert gqa["kernel_name"] == var["kernel_name"] == "tc_attn_kernel"
+    assert gqa["ctas"] <= gqa["num_sms"] and gqa["threads"] == 192
+    assert var["ctas"] > var["num_sms"] and var["threads"] == 320
+
+
 def test_plan_query_rejects_bad_arguments():
     _built()
     from cached_split_attention_b200 import binding as B
