@@ -76,6 +76,35 @@ def test_video_reduced_gamma_gate():
     assert any(r.recompute.any() and not r.recompute.all() for r in ref[1:])
 
 
+def _threads(w):
+    _, B = torch_and_binding()
+    return B.plan_query(B.DeviceProblem(w.problem, "cpu"))
+
+
+def test_tensor_core_two_threads_per_row_varlen():
+    """Grids of more than one wave run the tensor-core kernel with two softmax threads
+    per row (the halves of a row swap their maxima every chunk): ragged varlen
+    branches (prefix 300 + 37, chunks ending mid-way in both halves of a row), both
+    forced arms and the gate."""
+    w = W.varlen_branches(steps=4, prefix=337)
+    plan = _threads(w)
+    assert plan["kernel_name"] == "tc_attn_kernel" and plan["ctas"] > plan["num_sms"] and plan["threads"] == 320
+    _compare(w, flags=W.FORCE_RECOMPUTE)
+    _compare(w, flags=W.FORCE_REUSE)
+    _compare(w)
+
+
+def test_tensor_core_two_threads_per_row_gqa_locking():
+    """The same on a GQA batch of 40 sequences (320 groups, g = 4, half the block's
+    rows locked), whose reuse steps take the lean path with its loads after the
+    decision (the grid is more than one wave)."""
+    w = W.long_context_gqa(steps=3, batch=40, prefix=203)
+    plan = _threads(w)
+    assert plan["threads"] == 320 and plan["lean_reuse"] == 1 and plan["lean_early"] == 0
+    _compare(w, flags=W.FORCE_RECOMPUTE)
+    _compare(w, flags=W.FORCE_REUSE)
+
+
 def test_determinism():
     w = W.varlen_branches(steps=3, prefix=512)
     a, _ = run_policy_gpu(w)
