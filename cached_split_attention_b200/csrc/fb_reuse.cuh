@@ -105,14 +105,21 @@ __device__ __forceinline__ void lean_rows(int nrows, int split, int S, int& r0, 
   nr = min(nrows, (split + 1) * per * 16) - r0;
 }
 
-// Box token t has thread kLeanTok0 + t (warp 0 is left to the reuse decision's
-// loads); the host plan keeps bt <= threads - kLeanTok0.
+// Box token t has a thread of warps 1.. (warp 0 is left to the reuse decision's
+// loads), dealt round-robin over those warps so that each issues few of the
+// per-token copies (a warp issues its lanes' bulk copies one after another): token
+// t = lane * W + (warp - 1) with W = warps - 1.  The host plan keeps bt <= 32 W.
 constexpr int kLeanTok0 = 32;
+__device__ __forceinline__ int lean_tok(int tid) {
+  const int w1 = static_cast<int>(blockDim.x >> 5) - 1;
+  const int w = (tid >> 5) - 1;
+  return w < 0 ? -1 : (tid & 31) * w1 + w;
+}
 
 // Block position of the box token of thread `tid` (-1: none).  Read from q_rows
 // before the dependency wait; the caller has checked the sequence's ranges.
 __device__ __forceinline__ int lean_pos(const Params& p, int q0, const LeanRows& lr, int tid) {
-  const int t = tid - kLeanTok0;
+  const int t = lean_tok(tid);
   if (t < 0 || t >= lr.ntok) return -1;
   const int tok = lr.tok_lo + t;
   return p.q_rows ? p.q_rows[q0 + tok] : tok;
@@ -189,7 +196,7 @@ __device__ __forceinline__ void lean_fetch(const Params& p, const LeanSmem<D>& l
                                            int n_in, const LeanRows& lr, int pos, int tid) {
   const int g = p.g;
   if (tid == 0) mbar_arrive_expect_tx(&bars[1], lr.ntok * g * D * 4);
-  const int t = tid - kLeanTok0;
+  const int t = lean_tok(tid);
   if (t >= 0 && t < lr.ntok) {
     const bool good = pos >= 0 && pos < n_in;
     if (!good) record_status(kDevBadIndex);
