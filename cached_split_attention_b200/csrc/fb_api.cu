@@ -2,6 +2,7 @@
 // launch planning, the TMA descriptor cache and the kernel launches.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -23,6 +24,17 @@
 namespace {
 
 thread_local std::string t_err = "no error";
+
+// An NVTX range around one call that enqueues device work, named for the entry
+// point, so that a timeline tool shows where each call's launches were issued.
+// NVTX does nothing unless a tool is attached to the process.
+class Range {
+ public:
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 fb_status fail(fb_status s, const char* fmt, ...) {
   char buf[512];
@@ -464,6 +476,7 @@ fb_status fb_workspace_size(const fb_problem* problem, size_t* bytes) {
 }
 
 fb_status fb_workspace_init(void* workspace, size_t bytes, fb_stream_t stream) {
+  const Range range("fb_workspace_init");
   if (!workspace && bytes) return fail(FB_ERR_INVALID_ARG, "workspace is NULL");
   if (!bytes) return FB_OK;
   cudaError_t e = cudaMemsetAsync(workspace, 0, bytes, reinterpret_cast<cudaStream_t>(stream));
@@ -474,6 +487,7 @@ fb_status fb_workspace_init(void* workspace, size_t bytes, fb_stream_t stream) {
 fb_status fb_out_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16* k_out, const fb_bf16* v_out,
                       const uint8_t* head_mask, float* a_out, float* l_out, void* workspace, size_t workspace_bytes,
                       fb_stream_t stream) {
+  const Range range("fb_out_attn");
   FB_TRY(check_problem(problem));
   const bool rows = problem->total_q > 0;
   FB_TRY(check_ptr(q, "q", rows));
@@ -501,6 +515,7 @@ fb_status fb_out_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16
 
 fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16* k_in, const fb_bf16* v_in,
                      float* a_in, float* l_in, fb_stream_t stream) {
+  const Range range("fb_in_attn");
   FB_TRY(check_problem(problem));
   const bool rows = problem->total_q > 0;
   FB_TRY(check_ptr(q, "q", rows));
@@ -524,6 +539,7 @@ fb_status fb_in_attn(const fb_problem* problem, const fb_bf16* q, const fb_bf16*
 
 fb_status fb_merge(int64_t n, int32_t d, const float* a_out, const float* l_out, const float* a_in,
                    const float* l_in, float* a_full_f32, fb_bf16* a_full_bf16, float* l_full, fb_stream_t stream) {
+  const Range range("fb_merge");
   if (n < 0 || d <= 0) return fail(FB_ERR_INVALID_ARG, "n must be >= 0 and d > 0");
   if (n > INT64_MAX / d) return fail(FB_ERR_INVALID_ARG, "n x d overflows 64 bits");
   if (n == 0) return FB_OK;
@@ -540,6 +556,7 @@ fb_status fb_merge(int64_t n, int32_t d, const float* a_out, const float* l_out,
 
 fb_status fb_head_similarity(const fb_problem* problem, const fb_bf16* q, const fb_bf16* q_ref, float* cos_out,
                              fb_stream_t stream) {
+  const Range range("fb_head_similarity");
   FB_TRY(check_problem(problem));
   FB_TRY(check_ptr(q, "q", problem->total_q > 0));
   FB_TRY(check_ptr(q_ref, "q_ref", problem->total_kv_in > 0));
@@ -559,6 +576,7 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
                   const fb_bf16* k_in, const fb_bf16* v_in, const fb_bf16* k_out, const fb_bf16* v_out,
                   const int32_t* n_updated, const uint8_t* head_reuse_in, fb_bf16* a_full, float* l_full,
                   uint8_t* decision_out, void* workspace, size_t workspace_bytes, fb_stream_t stream) {
+  const Range range("fb_step");
   FB_TRY(check_problem(problem));
   if (!params) return fail(FB_ERR_INVALID_ARG, "params is NULL");
   if (!cache) return fail(FB_ERR_INVALID_ARG, "cache is NULL");
@@ -648,6 +666,7 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
 }
 
 fb_status fb_cache_invalidate(const fb_problem* problem, const fb_cache* cache, fb_stream_t stream) {
+  const Range range("fb_cache_invalidate");
   FB_TRY(check_problem(problem));
   if (!cache || (!cache->valid && problem->num_seqs > 0)) return fail(FB_ERR_INVALID_ARG, "cache->valid is NULL");
   const size_t n = static_cast<size_t>(problem->num_seqs) * problem->num_heads_q;
@@ -659,6 +678,7 @@ fb_status fb_cache_invalidate(const fb_problem* problem, const fb_cache* cache, 
 
 fb_status fb_cache_copy_seq(const fb_problem* problem, const fb_cache* cache, int32_t src_seq, int32_t dst_seq,
                             fb_stream_t stream) {
+  const Range range("fb_cache_copy_seq");
   FB_TRY(check_problem(problem));
   if (!cache) return fail(FB_ERR_INVALID_ARG, "cache is NULL");
   if (src_seq < 0 || src_seq >= problem->num_seqs || dst_seq < 0 || dst_seq >= problem->num_seqs)
@@ -681,6 +701,7 @@ fb_status fb_cache_copy_seq(const fb_problem* problem, const fb_cache* cache, in
 
 fb_status fb_cache_invalidate_seqs(const fb_problem* problem, const fb_cache* cache, const uint8_t* seq_mask,
                                    fb_stream_t stream) {
+  const Range range("fb_cache_invalidate_seqs");
   FB_TRY(check_problem(problem));
   if (!cache || (!cache->valid && problem->num_seqs > 0)) return fail(FB_ERR_INVALID_ARG, "cache->valid is NULL");
   if (problem->num_seqs == 0) return FB_OK;
@@ -696,6 +717,7 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
                            int32_t total_sel, const fb_bf16* k_out, const fb_bf16* v_out, const fb_bf16* k_in,
                            const fb_bf16* v_in, fb_bf16* k_ext, fb_bf16* v_ext, uint32_t* kv_out_skip,
                            int32_t* cu_seqlens_kv_in_ext, fb_stream_t stream) {
+  const Range range("fb_sparse_layout");
   FB_TRY(check_problem(problem));
   if (total_sel < 0 || total_sel > problem->total_kv_out)
     return fail(FB_ERR_INVALID_ARG, "total_sel %d outside [0, total_kv_out]", total_sel);
@@ -743,6 +765,7 @@ fb_status fb_sparse_layout(const fb_problem* problem, const int32_t* cu_sel, con
 fb_status fb_prefix_append(const fb_problem* problem, const fb_bf16* k_out, const fb_bf16* v_out,
                            const fb_bf16* k_in, const fb_bf16* v_in, fb_bf16* k_dst, fb_bf16* v_dst,
                            int32_t* cu_seqlens_kv_out_dst, fb_stream_t stream) {
+  const Range range("fb_prefix_append");
   FB_TRY(check_problem(problem));
   if (problem->num_seqs == 0) return FB_OK;
   if (problem->num_seqs > 65535)  // one grid row per sequence
@@ -785,6 +808,7 @@ fb_status fb_prefix_append(const fb_problem* problem, const fb_bf16* k_out, cons
 }
 
 fb_status fb_selftest_wait_timeout(fb_stream_t stream) {
+  const Range range("fb_selftest_wait_timeout");
   fb::wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "self-test kernel launch");
@@ -798,6 +822,7 @@ fb_status fb_release_cache(void) {
 }
 
 fb_status fb_device_status(int32_t* code, fb_stream_t stream) {
+  const Range range("fb_device_status");
   if (!code) return fail(FB_ERR_INVALID_ARG, "code is NULL");
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");

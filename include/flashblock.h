@@ -38,6 +38,11 @@
  *    seconds, records FB_ERR_TIMEOUT in a device status word and returns;
  *    fb_device_status() reads and clears it.  After a timeout the workspace
  *    must be re-initialised with fb_workspace_init().
+ *  - Tracing: every call that enqueues device work (fb_workspace_init, the
+ *    attention, merge, similarity, cache, layout and append calls, the
+ *    self-test and fb_device_status) opens an NVTX range named for itself on
+ *    entry and closes it on return, whatever it returns.  Without a tool
+ *    attached to the process NVTX does nothing.
  */
 #ifndef FLASHBLOCK_H
 #define FLASHBLOCK_H
