@@ -1,13 +1,13 @@
 """The lean reuse pass of fb_step against the oracle (needs a B200).
 
-On a reuse step of a block of at most 128 keys, the (sequence, kv-head) groups
-whose q-heads all reuse the cache are served by a short kernel that runs before
-the streaming kernel: block attention with warp MMA and the merge with the cached
-(A_out, L_out) rows (FlashBlock, "Mecanismo Central").  These cases put its edges
-under the same tolerances as every other step test: block lengths around the
-32-key slices and 64-key chunks (1 to 128 keys), head dims 64 and 128, grouped
-heads, a sequence with no active rows, locked rows, and calls in which some groups
-reuse while others recompute."""
+On a reuse step of a block of at most 128 keys, the work items (sequence,
+kv-head, row tile) whose q-heads all reuse the cache take the lean path inside
+the streaming kernels: block attention with warp MMA and the merge with the
+cached (A_out, L_out) rows (FlashBlock, "Mecanismo Central").  These cases put its
+edges under the same tolerances as every other step test: block lengths around
+the 32-key slices and 64-key chunks (1 to 128 keys), head dims 64 and 128, grouped
+heads up to the largest group the ABI takes (32), a sequence with no active rows,
+locked rows, and calls in which some groups reuse while others recompute."""
 import numpy as np
 import pytest
 
@@ -68,14 +68,24 @@ def test_block_lengths(block, d):
     assert ref[0].recompute.all() and not ref[1].recompute.any()
 
 
-@pytest.mark.parametrize("g", [2, 4, 8])
+@pytest.mark.parametrize("g", [2, 4, 8, 16, 32])
 def test_grouped_heads_locked_rows(g):
-    """GQA groups of g q-heads over 2 kv-heads; two sequences with locked rows
-    (active positions not the identity), blocks of 64 and 47 keys."""
+    """GQA groups of g q-heads over 2 kv-heads (tensor-core kernel, up to ten 128-row
+    tiles per group); two sequences with locked rows (active positions not the
+    identity), blocks of 64 and 47 keys."""
     rng = np.random.default_rng(g)
     active = [np.sort(rng.permutation(64)[:29]), np.sort(rng.permutation(47)[:40])]
     w = _workload([64, 47], active, 150, 2 * g, 2, 128)
     _compare(w, flags=W.FORCE_REUSE)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_largest_group_warp_mma(d):
+    """g = 32 with two active tokens per sequence: 64 rows per group, the warp-MMA
+    kernel's largest tile; ragged blocks of 8 and 5 keys, locked rows."""
+    w = _workload([8, 5], [np.array([1, 6]), np.array([0, 3])], 150, 64, 2, d)
+    ref = _compare(w, flags=W.FORCE_REUSE)
+    assert ref[0].recompute.all() and not ref[1].recompute.any()
 
 
 def test_sequence_without_active_rows():
@@ -87,8 +97,8 @@ def test_sequence_without_active_rows():
 
 def test_groups_reuse_and_recompute_in_one_call():
     """The tau gate per sequence and a caller mask per head: in the same call some
-    groups have every head reusing (served by the reuse pass) and others have at
-    least one head recomputing (served by the streaming kernel, all of their heads)."""
+    groups have every head reusing (served by the lean path) and others have at
+    least one head recomputing (streamed, all of their heads)."""
     w = _workload([64, 64, 64], [np.arange(64)] * 3, 200, 8, 2, 128, steps=4, redraw=3)
     for s, st in enumerate(w.steps[1:], start=1):   # sequence 1 passes tau = 4 on every step
         st.n_updated[:] = [3, 5, 2]
