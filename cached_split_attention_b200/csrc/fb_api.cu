@@ -620,7 +620,7 @@ fb_status fb_step(const fb_problem* problem, const fb_params* params, const fb_c
   FB_TRY(kv_map(k_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_k_in));
   FB_TRY(kv_map(v_in, problem->total_kv_in, problem->num_heads_kv, problem->head_dim, pl.bn, &prm.tm_v_in));
 
-  if (head_gate && rows) {
+  if (head_gate) {  // with no active rows every score is 0 (a zero denominator), never a stale one
     float* cos_ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_cos);
     FB_TRY(fb_head_similarity(problem, q, cache->q_ref, cos_ws, stream));
   }

@@ -68,7 +68,8 @@ typedef enum fb_status {
 
 /* Gate flags of fb_params.flags. */
 #define FB_GATE_TAU 1u        /* reuse only if n_updated[b] < tau (strict)               */
-#define FB_GATE_HEAD 2u       /* reuse head h only if cos(Q_bh, q_ref_bh) > gamma (strict) */
+#define FB_GATE_HEAD 2u       /* reuse head h only if cos(Q_bh, q_ref_bh) > gamma (strict);
+                                 a head with no active rows has cos 0                  */
 #define FB_FORCE_RECOMPUTE 4u /* recompute every head (dense step)                        */
 #define FB_FORCE_REUSE 8u     /* reuse every head whose cache is valid                    */
 /* Cumulative threshold gate: reuse only if cache->m_acc[b,h] + n_updated[b] < tau, i.e.

@@ -81,6 +81,67 @@ def _threads(w):
     return B.plan_query(B.DeviceProblem(w.problem, "cpu"))
 
 
+def _rows_vanish_workload(hq, hkv, blocks, prefix, flags, gamma, tau, seed=11):
+    """Two steps with every block row active, then two in which every row is locked
+    (the call has no query row at all): the gates still decide every head and the
+    cache state still moves.  The queries never change, so a head's cosine is 1
+    while it has rows."""
+    rng = np.random.default_rng(seed)
+    d = 128
+    p_all = W.make_problem([np.arange(B) for B in blocks], [prefix] * len(blocks), blocks, hq, hkv, d)
+    p_none = W.make_problem([np.zeros(0, np.int64) for _ in blocks], [prefix] * len(blocks), blocks, hq, hkv, d)
+    k_out = W.normal_bf16(rng, (p_all.total_kv_out, hkv, d))
+    v_out = W.normal_bf16(rng, (p_all.total_kv_out, hkv, d))
+    q_blk = W.normal_bf16(rng, (p_all.total_kv_in, hq, d))
+    k_blk = W.normal_bf16(rng, (p_all.total_kv_in, hkv, d))
+    v_blk = W.normal_bf16(rng, (p_all.total_kv_in, hkv, d))
+    n = np.ones(len(blocks), np.int32)
+    steps = [W.StepInput(q=q_blk.copy(), k_in=k_blk, v_in=v_blk, n_updated=n.copy(), problem=p_all)
+             for _ in range(2)]
+    steps += [W.StepInput(q=q_blk[:0].copy(), k_in=k_blk, v_in=v_blk, n_updated=n.copy(), problem=p_none)
+              for _ in range(2)]
+    return W.Workload("rows_vanish", p_all, k_out, v_out, steps, tau=tau, gamma=gamma, flags=flags)
+
+
+@pytest.mark.parametrize("flags", [W.GATE_HEAD, W.GATE_TAU, W.GATE_TAU_CUM, W.FORCE_REUSE, W.GATE_TAU | W.GATE_HEAD],
+                         ids=["gamma", "tau", "tau_cum", "force_reuse", "tau_and_gamma"])
+@pytest.mark.parametrize("hq,hkv,blocks", [(4, 4, (48, 29)), (8, 2, (32, 64))], ids=["warp_mma", "tensor_core"])
+def test_calls_with_no_active_rows(flags, hq, hkv, blocks):
+    """Degenerate calls (every row of every sequence locked) after calls with rows:
+    decisions, validity and the cumulative counts match the oracle.  With no rows a
+    head's cosine is 0 (a zero denominator), so the gamma gate recomputes; the score
+    is computed for the call, never left over from the previous one."""
+    w = _rows_vanish_workload(hq, hkv, list(blocks), 150, flags, gamma=0.5, tau=3)
+    gpu, cache = run_policy_gpu(w)
+    ocache = policy.OracleCache.empty(w.problem)
+    ref = policy.run_policy(w, cache=ocache)
+    for s, (g, r) in enumerate(zip(gpu, ref)):
+        assert np.array_equal(g["decision"], r.recompute), f"step {s}: decisions differ"
+        if r.a_full.shape[0]:
+            assert_close(g["a_full"], r.a_full, g["l_full"], r.l_full, f"step {s}")
+    S = w.problem.num_seqs
+    assert np.array_equal(cache.valid.cpu().numpy()[:S].astype(bool), ocache.valid)
+    assert np.array_equal(cache.m_acc.cpu().numpy()[:S], ocache.m_acc)
+    if flags & W.GATE_HEAD:
+        assert not ref[1].recompute.any() and ref[2].recompute.all()
+
+
+@pytest.mark.parametrize("make", [
+    lambda: W.dllm_layer(steps=4, prefix=2000, heads=8),
+    lambda: W.dllm_layer(steps=4, prefix=2000, heads=8, head_dim=64),
+    lambda: W.long_context_gqa(steps=3, batch=1, prefix=2085),
+], ids=["warp_mma_d128", "warp_mma_d64", "tensor_core"])
+def test_eight_cta_clusters(make):
+    """Few groups on a long prefix: the plan splits every group's prefix over the
+    largest portable cluster (8 CTAs), so the log-space combine reads seven remote
+    partials through distributed shared memory; ragged last chunks; the forced
+    recompute arm and the workload's own gates (reuse steps on the lean path)."""
+    w = make()
+    assert _threads(w)["splits"] == 8
+    _compare(w, flags=W.FORCE_RECOMPUTE)
+    _compare(w)
+
+
 def test_tensor_core_two_threads_per_row_varlen():
     """Grids of more than one wave run the tensor-core kernel with two softmax threads
     per row (the halves of a row swap their maxima every chunk): ragged varlen
