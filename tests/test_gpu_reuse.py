@@ -88,6 +88,17 @@ def test_largest_group_warp_mma(d):
     assert ref[0].recompute.all() and not ref[1].recompute.any()
 
 
+@pytest.mark.parametrize("hq,hkv,d", [(4, 4, 64), (8, 2, 128)], ids=["warp_mma", "tensor_core"])
+def test_no_prefix_at_all(hq, hkv, d):
+    """Every sequence has an empty prefix (J_out empty, so the cached partial is
+    (0, -inf) and the merge gives the block partial itself): both forced arms and
+    the tau gate."""
+    w = _workload([40, 29], [np.arange(40), np.arange(3, 29, 2)], 0, hq, hkv, d)
+    _compare(w, flags=W.FORCE_RECOMPUTE)
+    _compare(w, flags=W.FORCE_REUSE)
+    _compare(w)
+
+
 def test_sequence_without_active_rows():
     """A sequence whose rows are all locked has nothing to write; its neighbours
     reuse normally."""
