@@ -126,6 +126,25 @@ def test_calls_with_no_active_rows(flags, hq, hkv, blocks):
         assert not ref[1].recompute.any() and ref[2].recompute.all()
 
 
+@pytest.mark.parametrize("arm", ["tau", "gamma", "recompute", "reuse"])
+def test_two_tile_sequences_with_one_and_no_rows(arm):
+    """Two-tile kernel (one q-head per kv-head, a 300-row sequence) in a call that
+    also holds a sequence with a single active row and one whose rows are all
+    locked: work items with one row and an empty second tile, and items with no row
+    at all; under the similarity gate the heads decide differently per sequence and
+    the work-order pass puts the recomputing items first."""
+    import dataclasses
+    from test_gpu_reuse import _workload
+    w = _workload([300, 40, 24], [np.arange(300), np.array([7]), np.zeros(0, np.int64)], 200, 2, 2, 128, steps=4)
+    assert _threads(w)["kernel_name"] == "tc2_attn_kernel"
+    flags = {"tau": None, "gamma": None, "recompute": W.FORCE_RECOMPUTE, "reuse": W.FORCE_REUSE}[arm]
+    if arm == "gamma":
+        w = dataclasses.replace(w, gamma=0.5, flags=W.GATE_HEAD | W.GATE_TAU)
+    _, ref = _compare(w, flags=flags)
+    if arm == "gamma":
+        assert all(not r.recompute[0].any() and r.recompute[1:].all() for r in ref[1:])
+
+
 @pytest.mark.parametrize("make", [
     lambda: W.dllm_layer(steps=4, prefix=2000, heads=8),
     lambda: W.dllm_layer(steps=4, prefix=2000, heads=8, head_dim=64),
