@@ -227,6 +227,35 @@ def test_plan_query_tensor_core_threads_per_row():
     assert var["ctas"] > var["num_sms"] and var["threads"] == 320
 
 
+def test_plan_query_reaches_the_variants_the_gpu_tests_name():
+    """The reduced shapes of the GPU tests reach the launch variants those tests are
+    named for (so that a change of the host plan shows up here, without a GPU): the
+    largest portable cluster on both streaming kernels, the largest group (32 q-heads
+    per kv-head) on both, the two-tile kernel with one-row and empty sequences, and
+    the warp-MMA kernel for a call whose rows are all locked."""
+    _built()
+    from cached_split_attention_b200 import binding as B
+    from cached_split_attention_b200 import workloads as W
+    mk = W.make_problem
+    none = np.zeros(0, np.int64)
+    cases = [
+        # (problem, kernel, threads, splits or None)
+        (W.dllm_layer(steps=1, prefix=2000, heads=8).problem, "attn_kernel", 256, 8),
+        (W.dllm_layer(steps=1, prefix=2000, heads=8, head_dim=64).problem, "attn_kernel", 256, 8),
+        (W.long_context_gqa(steps=1, batch=1, prefix=2085).problem, "tc_attn_kernel", 192, 8),
+        (mk([np.arange(29), np.arange(40)], [150, 150], [64, 47], 64, 2, 128), "tc_attn_kernel", 192, None),
+        (mk([np.array([1, 6]), np.array([0, 3])], [150, 150], [8, 5], 64, 2, 128), "attn_kernel", 256, None),
+        (mk([np.arange(300), np.array([7]), none], [200] * 3, [300, 40, 24], 2, 2, 128), "tc2_attn_kernel", 320, 1),
+        (mk([none, none], [150, 150], [32, 64], 8, 2, 128), "attn_kernel", 128, None),
+        (W.varlen_branches(steps=1, prefix=337).problem, "tc_attn_kernel", 320, None),
+    ]
+    for p, kernel, threads, splits in cases:
+        info = B.plan_query(B.DeviceProblem(p, "cpu"))
+        assert (info["kernel_name"], info["threads"]) == (kernel, threads), info
+        if splits is not None:
+            assert info["splits"] == splits, info
+
+
 def test_plan_query_rejects_bad_arguments():
     _built()
     from cached_split_attention_b200 import binding as B
